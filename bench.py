@@ -1,0 +1,362 @@
+#!/usr/bin/env python
+"""Benchmark: indexed sparse decode at 128K context, M = 2048 (queries/s and HBM roofline).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--batch B]
+
+Workload (one step = one decode token for every sequence of the batch, whole path):
+B = 16 sequences, 64 query heads / 8 KV heads, d = 128, n = 131072 cached tokens,
+r = 32 FP8 projected keys, M = 2048, bf16 paged KV cache (page 64, random page table).
+Inputs are seeded synthetic data resident in HBM; they touch ~671 MB per step, well
+above the 126 MB L2, so no L2 flush is used between steps.
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
+data path); the time is the max over ranks.  --impl reference times the fp64 CPU oracle
+on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-decode attn queries/sec at 128K ctx, M=2048; achieved HBM GB/s vs peak"
+WORKLOAD = "128K paged decode: B=16, 64q/8kv heads, d=128, n=131072, r=32 FP8 projected keys, M=2048, page 64"
+FALLBACK_HBM_GBS = 6650.0
+INDEX_SOURCES = ["indexed_top_sparse_b200/csrc/lisa_index.cu", "indexed_top_sparse_b200/csrc/lisa_common.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "index_select_128k_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--batch", type=int, default=16, help="sequences per GPU (16 = the workload; smaller for profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline sample budget")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the index kernel from the committed ncu summary, if still current."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("source_hash") == source_hash(INDEX_SOURCES):
+            return float(t["dram_bytes_per_launch_full_workload"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def oracle_sample(prob_host_fn, budget_s: float):
+    """Time the oracle on whole queries (one sequence, all KV heads) until budget_s is spent."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle import lisa_oracle as O
+
+    done, t_total, samples = 0, 0.0, []
+    with threadpool_limits(limits=1):
+        while t_total < budget_s and done < 64:
+            inp = prob_host_fn(done)
+            t0 = time.perf_counter()
+            O.decode_step(inp)
+            dt = time.perf_counter() - t0
+            samples.append(dt)
+            t_total += dt
+            done += 1
+    return done, t_total
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 CPU oracle, as it stands, on sampled queries of the same workload."""
+    if rank != 0:
+        return
+    from workloads import config3
+    from workloads.host_view import host_inputs
+
+    # One sequence of the workload per sample, drawn on the CPU (same shapes and recipe).
+    def sample(i):
+        return host_inputs(config3(device="cpu", B=1, seed=2000 + i))
+
+    inputs = [sample(i) for i in range(min(2, args.steps + args.warmup))]
+    from threadpoolctl import threadpool_limits
+
+    from oracle import lisa_oracle as O
+
+    times = []
+    with threadpool_limits(limits=1):
+        for k in range(args.warmup + args.steps):
+            inp = inputs[k % len(inputs)]
+            t0 = time.perf_counter()
+            O.decode_step(inp)
+            if k >= args.warmup:
+                times.append(time.perf_counter() - t0)
+    per_query = sum(times) / len(times)
+    value = 1.0 / per_query
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_query * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "step": "one query (1 sequence, 8 KV heads) per step, fp64 oracle"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{args.steps} timed queries of the 128K workload, one sequence each"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import indexed_top_sparse_b200 as L
+    from workloads import config3
+    from workloads import run as R
+    from workloads.host_view import host_inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    prob = config3(device=dev, B=args.batch, seed=1003 + rank)
+    desc = R.desc_of(prob)
+    ws = L.alloc_workspace(desc, dev)
+    B, Hq, d = prob.B, prob.Hq, prob.d
+    out = torch.empty(B, Hq, d, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    scale = prob.kproj_scale.to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None, q=None):
+        L.lisa_fused_decode(desc, prob.q if q is None else q, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale,
+                            prob.k_pool, prob.v_pool, None, None, None, None, None, out, lse, ws, events=events,
+                            stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if L.lisa_check_device_error(ws) != 0:
+        raise RuntimeError("device range check failed on the benchmark workload")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    stage = [L.stage_events(*e) for e in evs]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for k in range(K):
+            step(stage[k])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = t0.elapsed_time(t1)
+    idx_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    attn_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    merge_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / K
+
+    # End to end through the same entry point: q from pinned host memory in, out back to pinned host memory.
+    q_host = prob.q.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    q_dev = torch.empty_like(prob.q)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K2 = max(1, min(K, 100))
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K2):
+        q_dev.copy_(q_host, non_blocking=True)
+        step(q=q_dev)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / K2
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    flags = L.lisa_check_device_error(ws)
+
+    if rank != 0:
+        return
+    req = prob.required_bytes_per_query()
+    step_bytes = float(sum(req))
+    kproj_bytes = float(sum(int(n) * prob.r * prob.Hkv for n in prob.seq_lens.tolist()))
+    hbm, hbm_kind = peaks()
+    achieved = kproj_bytes / (idx_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": B * world / (ms_step * 1e-3),
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8e4m3+bf16 in, fp32 accumulate",
+        "data": "synthetic",
+        "config": {
+            "workload": WORKLOAD if args.batch == 16 else WORKLOAD.replace("B=16", f"B={args.batch}"),
+            "sequences_per_gpu": B,
+            "l2": "inputs larger than L2 (~671 MB touched per step, 126 MB L2); no flush",
+            "launch": "lisa_fused_decode per step (index+select, split attention, merge)",
+        },
+        "roofline": {
+            "kernel": "lisa_index_select_kernel (FP8 score + cluster top-M)",
+            "bound": "hbm",
+            "achieved": achieved,
+            "peak": hbm,
+            "peak_kind": f"{hbm_kind} hbm_gbs" + (" (MEASURED_PEAKS.json)" if hbm_kind == "measured" else ""),
+            "unit": "GB/s",
+            "frac": achieved / hbm,
+            "traffic": recorded_traffic(),
+            "algorithmic_bytes_per_launch": kproj_bytes,
+            "avg_launch_ms": idx_ms,
+        },
+        "path_roofline": {
+            "required_bytes_per_step": step_bytes,
+            "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+            "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm,
+            "stage_ms": {"index_select": idx_ms, "attention": attn_ms, "merge": merge_ms},
+        },
+        "e2e": {
+            "value": B * world / (e2e_ms * 1e-3),
+            "unit": "queries/s",
+            "h2d_bytes_per_step": int(prob.q.numel() * 2),
+            "d2h_bytes_per_step": int(out.numel() * 2),
+        },
+        "gpu_launches": 3 * K,
+        "clocks": clk.summary(),
+        "device_check_flags": flags,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        def sample(i):
+            return host_inputs(prob, seqs=[i % B])
+
+        nq, secs = oracle_sample(sample, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": nq / secs, "unit": "queries/s", "cores": 1, "kind": "oracle",
+            "sample": f"{nq} queries (whole sequences, all 8 KV heads) of this workload, fp64 numpy, 1 thread",
+        }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = (1, 0, 0)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+/*
+ * lisa.h -- C ABI of the B200 (sm_100a) indexed sparse decode-attention library.
+ *
+ * One decode step for a batch of sequences, per KV head h of sequence b:
+ *
+ *   1. qbar  = mean of the G = Hq/Hkv query vectors of KV head h          (query head j -> KV head j / G)
+ *   2. u     = P_h qbar                       (P_h: r x d basis, caller supplied)
+ *   3. s_t   = scale_h * <u, c_t>   for every cached position t < n_b   (c_t: projected key, FP8 E4M3 or fp32)
+ *   4. I     = the min(M, n_b) positions of largest s_t; a tie at the M-th score goes to the lower position;
+ *              reported in ascending position order
+ *   5. o_j   = softmax attention of query head j over the bf16 keys/values of the positions in I, read
+ *              straight from the paged KV cache (no gathered copy)
+ *   6. (optional) linear branch:  S += phi(k_new) v_new^T,  z += phi(k_new),  lin_j = phi(q_j)^T S / (phi(q_j).z),
+ *              phi = elu + 1, and out_j = sigmoid(g_j) o_j + (1 - sigmoid(g_j)) lin_j
+ *   7. (optional) cross-layer reuse: a layer may take I from an earlier layer instead of steps 1-4.
+ *
+ * Sources.  Steps 1-5: JSSA write-up (rit.work, "jssa-sparse-attention-long-context"; article "Joint
+ * Subspace Sparse Attention for Efficient Long-Context Decoding"), section "Как JSSA сохраняет порядок
+ * токенов": queries of one KV head are averaged, projected into the head's joint subspace and every
+ * position is scored against an FP8 projected-key cache; attention is then exact over the original
+ * full-size keys and values; each GQA group keeps its own index set and one kernel launch reads the
+ * selected positions of all heads directly from the cache.  Step 6: LISA write-ups (aikraft.ru, section
+ * "Архитектура LISA"; opennieuws.be, section "Hybride architectuur voor efficiëntie"): a linear-attention
+ * branch beside the top-M sparse branch, fused by a gate.  Step 7: IndexCache write-up
+ * (denisavetisyan.com, section "IndexCache: Совместное использование слоев ..."): Shared layers reuse
+ * the indices of the preceding Full layer.  Where the pages leave a step open (scale, FP8 variant, tie
+ * rule, phi, gate form) the plain reading above is used.
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers (memory of the current CUDA device), allocated and owned
+ *     by the caller; the library never allocates or frees, and keeps no state between calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and runs
+ *     asynchronously; no entry point synchronises the host except lisa_check_device_error.
+ *   - Arguments are checked on the host before anything is enqueued.  Any return other than LISA_OK
+ *     from the checks means nothing was enqueued.  A failed launch returns LISA_ERR_CUDA.
+ *   - Values that can only be checked on the device (sequence lengths, page ids, indices, counts) are
+ *     checked by the kernels: an out-of-range value is clamped to a safe one, the computation goes on,
+ *     and a sticky bit is set in the workspace error word, read by lisa_check_device_error.
+ *   - `ws` is a caller-owned device workspace of at least lisa_workspace_size(desc) bytes, 256-byte
+ *     aligned, zeroed once with lisa_workspace_init before first use.  Its first 256 bytes hold the
+ *     error word; the rest is scratch.  Calls that share one workspace must not overlap in time.
+ *
+ * Layouts (row-major, innermost index last):
+ *   q            bf16 [B][Hq][d]
+ *   P            fp32 [Hkv][r][d]
+ *   kproj_pool   [num_pages][Hkv][page_size][r]  of uint8 E4M3 codes, or of fp32
+ *   kproj_scale  fp32 [Hkv]
+ *   k_pool/v_pool bf16 [num_pages][page_size][Hkv][d]
+ *   page_table   int32 [B][max_pages_per_seq]: position t of sequence b lives in page page_table[b][t /
+ *                page_size], slot t % page_size.  A contiguous cache is a pool with an identity table.
+ *   seq_lens     int32 [B], 0 <= n_b <= max_seq_len
+ *   scores       fp32 [B][Hkv][max_seq_len]
+ *   idx          int32 [B][Hkv][M], count int32 [B][Hkv]
+ *   out          bf16 [B][Hq][d],   lse fp32 [B][Hq] (natural log of the softmax denominator)
+ *
+ * Supported shapes (anything else returns LISA_ERR_UNSUPPORTED): d in {64, 128}; r in {16, 32};
+ * 1 <= G <= 8; page_size a power of two in [16, 1024]; 1 <= M <= 16384; max_seq_len <= 262144.
+ */
+#ifndef LISA_H
+#define LISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lisa_stream_t; /* same type as cudaStream_t */
+typedef struct CUevent_st* lisa_event_t;   /* same type as cudaEvent_t */
+
+typedef enum {
+  LISA_OK = 0,
+  LISA_ERR_INVALID_ARG = 1,  /* null pointer where one is required, negative size, inconsistent sizes */
+  LISA_ERR_UNSUPPORTED = 2,  /* valid but outside the supported shapes listed above */
+  LISA_ERR_WORKSPACE = 3,    /* ws is NULL, misaligned or smaller than lisa_workspace_size() */
+  LISA_ERR_CUDA = 4,         /* a CUDA call failed (launch or attribute query) */
+  LISA_ERR_DEVICE_CHECK = 5, /* lisa_check_device_error found a device-side range violation */
+  LISA_ERR_TIMEOUT = 6       /* reserved: a bounded device wait ran out (no current kernel waits) */
+} lisa_status;
+
+typedef enum { LISA_KPROJ_FP32 = 0, LISA_KPROJ_FP8_E4M3 = 1 } lisa_kproj_dtype;
+
+/* Device error word bits (lisa_check_device_error). */
+#define LISA_DEVERR_SEQ_LEN 0x1u    /* seq_lens[b] < 0 or > max_seq_len (clamped)                */
+#define LISA_DEVERR_PAGE_ID 0x2u    /* page id outside [0, num_pages) (row 0 of the pool used)   */
+#define LISA_DEVERR_INDEX 0x4u      /* idx entry outside [0, n_b) (position 0 used)              */
+#define LISA_DEVERR_COUNT 0x8u      /* count[b][h] outside [0, min(M, n_b)] (clamped)            */
+
+/* Sizes and the two caller-owned tables of one decode step.  Plain data; no ownership taken. */
+typedef struct {
+  int32_t batch;             /* B >= 0 (B = 0: every entry point returns LISA_OK and does nothing) */
+  int32_t num_q_heads;       /* Hq, a multiple of num_kv_heads                                     */
+  int32_t num_kv_heads;      /* Hkv >= 1                                                           */
+  int32_t head_dim;          /* d                                                                  */
+  int32_t idx_dim;           /* r, projected-key width                                             */
+  int32_t budget_m;          /* M, index-set size per (b, KV head)                                 */
+  int32_t page_size;         /* tokens per page                                                    */
+  int32_t max_pages_per_seq; /* columns of page_table, >= ceil(max_seq_len / page_size)            */
+  int32_t max_seq_len;       /* upper bound of seq_lens; row stride of `scores`                    */
+  int32_t num_pages;         /* pages in each pool (bounds for page ids)                          */
+  const int32_t* seq_lens;   /* device int32 [B]                                                   */
+  const int32_t* page_table; /* device int32 [B][max_pages_per_seq]                                */
+  float softmax_scale;       /* attention logit scale; <= 0 selects 1/sqrt(d)                      */
+} lisa_decode_desc;
+
+/* Optional linear-attention branch (one state per (b, KV head)); S and z are updated in place. */
+typedef struct {
+  float* S;                 /* device fp32 [B][Hkv][d][d]                     */
+  float* z;                 /* device fp32 [B][Hkv][d]                        */
+  const void* k_new;        /* device bf16 [B][Hkv][d], key of the new token  */
+  const void* v_new;        /* device bf16 [B][Hkv][d]                        */
+  const float* gate_logit;  /* device fp32 [Hq], g_j                          */
+} lisa_linear_branch;
+
+/* Optional events recorded on `stream` between the stages of lisa_fused_decode (any may be NULL). */
+typedef struct {
+  lisa_event_t start;       /* before the index stage (score + top-M)         */
+  lisa_event_t after_index; /* after the index stage, before attention        */
+  lisa_event_t after_attn;  /* after the split attention, before the merge    */
+  lisa_event_t end;         /* after the merge / linear branch / gate         */
+} lisa_stage_events;
+
+/* Workspace bytes any entry point needs for `desc` (0 if desc is invalid). Host only. */
+size_t lisa_workspace_size(const lisa_decode_desc* desc);
+
+/* Number of attention partitions per (b, KV head) the library uses for `desc` (0 if invalid). */
+int32_t lisa_num_splits(const lisa_decode_desc* desc);
+
+/* Zero the workspace error word (enqueued on stream). Call once after allocating ws. */
+lisa_status lisa_workspace_init(void* ws, size_t ws_bytes, lisa_stream_t stream);
+
+/* Steps 1-3: write s_t to scores[b][h][t] for t < n_b (entries t >= n_b are not written). */
+lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const float* P,
+                             const void* kproj_pool, lisa_kproj_dtype kproj_dtype,
+                             const float* kproj_scale, float* scores, void* ws, size_t ws_bytes,
+                             lisa_stream_t stream);
+
+/* Step 4 from caller-given fp32 scores: idx[b][h][0..count) ascending, count = min(M, n_b),
+ * idx[b][h][count..M) = -1. */
+lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx,
+                             int32_t* count, void* ws, size_t ws_bytes, lisa_stream_t stream);
+
+/* Steps 1-4 fused: the scores never leave on-chip memory. Same outputs as lisa_topm_select. */
+lisa_status lisa_index_topm(const lisa_decode_desc* desc, const void* q, const float* P,
+                            const void* kproj_pool, lisa_kproj_dtype kproj_dtype,
+                            const float* kproj_scale, int32_t* idx, int32_t* count, void* ws,
+                            size_t ws_bytes, lisa_stream_t stream);
+
+/* Step 5 over a caller-given index set (positions idx[b][h][0..count[b][h]) of sequence b).
+ * lse may be NULL. */
+lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q, const void* k_pool,
+                                    const void* v_pool, const int32_t* idx, const int32_t* count,
+                                    void* out, float* lse, void* ws, size_t ws_bytes,
+                                    lisa_stream_t stream);
+
+/* Steps 1-7 in one call.  reuse_idx/reuse_count (both or neither): take the index set from an
+ * earlier layer and skip steps 1-4 (kproj_pool, P, kproj_scale may then be NULL).  idx_out/count_out
+ * (both or neither, only without reuse): also return the index set.  lin may be NULL (no linear
+ * branch).  lse and events may be NULL. */
+lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const float* P,
+                              const void* kproj_pool, lisa_kproj_dtype kproj_dtype,
+                              const float* kproj_scale, const void* k_pool, const void* v_pool,
+                              const int32_t* reuse_idx, const int32_t* reuse_count, int32_t* idx_out,
+                              int32_t* count_out, const lisa_linear_branch* lin, void* out,
+                              float* lse, void* ws, size_t ws_bytes,
+                              const lisa_stage_events* events, lisa_stream_t stream);
+
+/* Synchronise `stream`, read the workspace error word into *flags_out (may be NULL), clear it.
+ * Returns LISA_ERR_DEVICE_CHECK if any bit was set, LISA_OK otherwise. */
+lisa_status lisa_check_device_error(void* ws, uint32_t* flags_out, lisa_stream_t stream);
+
+/* Static description of a status code. */
+const char* lisa_status_string(lisa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LISA_H */

@@ -1,0 +1,371 @@
+// C ABI of the indexed sparse decode library: argument checks, workspace layout, launches.
+// The operations and their sources are described in include/lisa.h.
+
+#include <math.h>
+
+#include "lisa.h"
+#include "lisa_common.cuh"
+#include "lisa_kernels.h"
+
+namespace {
+
+using namespace lisa;
+
+constexpr int kTargetAttnCtas = 148 * 2 * 4;  // SMs x resident CTAs x waves worth of partitions
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+inline int ilog2(int x) {
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return l;
+}
+
+struct Layout {
+  int G = 0, splits = 0, split_len = 0, chunk_max = 0;
+  size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0, total = 0;
+};
+
+// Host checks shared by every entry point.  Returns LISA_OK for a valid desc (also when B == 0).
+lisa_status check_desc(const lisa_decode_desc* d) {
+  if (d == nullptr) return LISA_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->head_dim <= 0 || d->budget_m <= 0 ||
+      d->page_size <= 0 || d->max_pages_per_seq <= 0 || d->max_seq_len <= 0 || d->num_pages <= 0)
+    return LISA_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return LISA_ERR_INVALID_ARG;
+  if ((long long)d->max_pages_per_seq * d->page_size < d->max_seq_len) return LISA_ERR_INVALID_ARG;
+  if (d->batch > 0 && (d->seq_lens == nullptr || d->page_table == nullptr)) return LISA_ERR_INVALID_ARG;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (G > kMaxG) return LISA_ERR_UNSUPPORTED;
+  if (d->head_dim != 64 && d->head_dim != 128) return LISA_ERR_UNSUPPORTED;
+  if (!is_pow2(d->page_size) || d->page_size < 16 || d->page_size > 1024) return LISA_ERR_UNSUPPORTED;
+  if (d->budget_m > kMaxBudget || d->max_seq_len > kMaxSeqLen) return LISA_ERR_UNSUPPORTED;
+  if (d->batch > 65535 || d->num_kv_heads > 65535) return LISA_ERR_UNSUPPORTED;
+  if ((unsigned long long)d->num_pages * (unsigned long long)d->page_size * (unsigned long long)d->num_kv_heads >
+      0xffffffffull)
+    return LISA_ERR_UNSUPPORTED;
+  return LISA_OK;
+}
+
+lisa_status check_idx_dim(const lisa_decode_desc* d) {
+  return (d->idx_dim == 16 || d->idx_dim == 32) ? LISA_OK : LISA_ERR_UNSUPPORTED;
+}
+
+Layout layout_of(const lisa_decode_desc& d) {
+  Layout L;
+  L.G = d.num_q_heads / d.num_kv_heads;
+  const int tiles = (d.budget_m + kAttnTile - 1) / kAttnTile;
+  const int pairs = d.batch > 0 ? d.batch * d.num_kv_heads : 1;
+  int splits = (kTargetAttnCtas + pairs - 1) / pairs;
+  const int min_splits = (d.budget_m + kMaxSplitLen - 1) / kMaxSplitLen;
+  if (splits < min_splits) splits = min_splits;
+  if (splits > tiles) splits = tiles;
+  L.split_len = ((tiles + splits - 1) / splits) * kAttnTile;
+  L.splits = (d.budget_m + L.split_len - 1) / L.split_len;
+  const int per_cta = (d.max_seq_len + kClusterSize - 1) / kClusterSize;
+  L.chunk_max = ((per_cta + d.page_size - 1) / d.page_size) * d.page_size;
+  const size_t B = (size_t)d.batch, Hkv = (size_t)d.num_kv_heads;
+  size_t off = kErrBytes;
+  L.off_idx = off;
+  off += align256(B * Hkv * (size_t)d.budget_m * 4);
+  L.off_count = off;
+  off += align256(B * Hkv * 4);
+  L.off_opart = off;
+  off += align256(B * Hkv * (size_t)L.splits * L.G * (size_t)d.head_dim * 4);
+  L.off_ml = off;
+  off += align256(B * Hkv * (size_t)L.splits * L.G * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+lisa_status check_ws(const void* ws, size_t bytes, const Layout& L) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < L.total) return LISA_ERR_WORKSPACE;
+  return LISA_OK;
+}
+
+// Make the device that owns `ptr` current for this library's CUDA runtime.
+lisa_status bind_device(const void* ptr) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return LISA_ERR_CUDA;
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return LISA_ERR_INVALID_ARG;
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return LISA_ERR_CUDA;
+  if (cur != a.device && cudaSetDevice(a.device) != cudaSuccess) return LISA_ERR_CUDA;
+  return LISA_OK;
+}
+
+inline lisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LISA_OK : LISA_ERR_CUDA; }
+
+// Pointers read with 16-byte vector loads or cp.async must be 16-byte aligned.
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
+  IndexParams p{};
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.d = d.head_dim;
+  p.r = d.idx_dim;
+  p.M = d.budget_m;
+  p.ps = d.page_size;
+  p.log2ps = ilog2(d.page_size);
+  p.max_pages = d.max_pages_per_seq;
+  p.max_seq_len = d.max_seq_len;
+  p.num_pages = d.num_pages;
+  p.chunk_max = L.chunk_max;
+  p.seq_lens = d.seq_lens;
+  p.page_table = d.page_table;
+  p.err = static_cast<uint32_t*>(ws);
+  return p;
+}
+
+AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, const void* q, const void* k_pool,
+                       const void* v_pool, const int32_t* idx, const int32_t* count) {
+  AttnParams p{};
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.d = d.head_dim;
+  p.M = d.budget_m;
+  p.ps = d.page_size;
+  p.log2ps = ilog2(d.page_size);
+  p.max_pages = d.max_pages_per_seq;
+  p.max_seq_len = d.max_seq_len;
+  p.num_pages = d.num_pages;
+  p.splits = L.splits;
+  p.split_len = L.split_len;
+  const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.seq_lens = d.seq_lens;
+  p.page_table = d.page_table;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k_pool = static_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = static_cast<const __nv_bfloat16*>(v_pool);
+  p.idx = idx;
+  p.count = count;
+  char* w = static_cast<char*>(ws);
+  p.o_part = reinterpret_cast<float*>(w + L.off_opart);
+  p.ml_part = reinterpret_cast<float*>(w + L.off_ml);
+  p.err = static_cast<uint32_t*>(ws);
+  return p;
+}
+
+MergeParams merge_params(const lisa_decode_desc& d, const Layout& L, void* ws, const void* q, void* out, float* lse,
+                         const lisa_linear_branch* lin) {
+  MergeParams m{};
+  m.B = d.batch;
+  m.Hq = d.num_q_heads;
+  m.Hkv = d.num_kv_heads;
+  m.d = d.head_dim;
+  m.splits = L.splits;
+  char* w = static_cast<char*>(ws);
+  m.o_part = reinterpret_cast<const float*>(w + L.off_opart);
+  m.ml_part = reinterpret_cast<const float*>(w + L.off_ml);
+  m.q = static_cast<const __nv_bfloat16*>(q);
+  m.out = static_cast<__nv_bfloat16*>(out);
+  m.lse = lse;
+  if (lin != nullptr) {
+    m.S = lin->S;
+    m.z = lin->z;
+    m.k_new = static_cast<const __nv_bfloat16*>(lin->k_new);
+    m.v_new = static_cast<const __nv_bfloat16*>(lin->v_new);
+    m.gate = lin->gate_logit;
+  }
+  return m;
+}
+
+lisa_status record(lisa_event_t ev, cudaStream_t stream) {
+  if (ev == nullptr) return LISA_OK;
+  return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), stream));
+}
+
+#define LISA_TRY(expr)                  \
+  do {                                  \
+    const lisa_status _s = (expr);      \
+    if (_s != LISA_OK) return _s;       \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t lisa_workspace_size(const lisa_decode_desc* desc) {
+  if (check_desc(desc) != LISA_OK) return 0;
+  return layout_of(*desc).total;
+}
+
+int32_t lisa_num_splits(const lisa_decode_desc* desc) {
+  if (check_desc(desc) != LISA_OK) return 0;
+  return layout_of(*desc).splits;
+}
+
+lisa_status lisa_workspace_init(void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  if (ws == nullptr || ws_bytes < kErrBytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return LISA_ERR_WORKSPACE;
+  LISA_TRY(bind_device(ws));
+  return cuda_status(cudaMemsetAsync(ws, 0, kErrBytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,
+                             lisa_kproj_dtype kproj_dtype, const float* kproj_scale, float* scores, void* ws,
+                             size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  LISA_TRY(check_idx_dim(desc));
+  if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || scores == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
+  if (!aligned16(kproj_pool) || !aligned4(q) || !aligned4(scores)) return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  IndexParams p = index_params(*desc, L, ws);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.P = P;
+  p.kproj = kproj_pool;
+  p.kproj_fp8 = kproj_dtype == LISA_KPROJ_FP8_E4M3;
+  p.kproj_scale = kproj_scale;
+  p.scores = scores;
+  return cuda_status(launch_index_score(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx, int32_t* count,
+                             void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  if (scores == nullptr || idx == nullptr || count == nullptr) return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  IndexParams p = index_params(*desc, L, ws);
+  p.scores = const_cast<float*>(scores);
+  p.idx = idx;
+  p.count = count;
+  return cuda_status(launch_index_select(p, true, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_index_topm(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,
+                            lisa_kproj_dtype kproj_dtype, const float* kproj_scale, int32_t* idx, int32_t* count,
+                            void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  LISA_TRY(check_idx_dim(desc));
+  if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || idx == nullptr ||
+      count == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
+  if (!aligned16(kproj_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  IndexParams p = index_params(*desc, L, ws);
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.P = P;
+  p.kproj = kproj_pool;
+  p.kproj_fp8 = kproj_dtype == LISA_KPROJ_FP8_E4M3;
+  p.kproj_scale = kproj_scale;
+  p.idx = idx;
+  p.count = count;
+  return cuda_status(launch_index_select(p, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q, const void* k_pool,
+                                    const void* v_pool, const int32_t* idx, const int32_t* count, void* out,
+                                    float* lse, void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || idx == nullptr || count == nullptr || out == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LISA_TRY(cuda_status(launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count), st)));
+  return cuda_status(launch_merge(merge_params(*desc, L, ws, q, out, lse, nullptr), st));
+}
+
+lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,
+                              lisa_kproj_dtype kproj_dtype, const float* kproj_scale, const void* k_pool,
+                              const void* v_pool, const int32_t* reuse_idx, const int32_t* reuse_count,
+                              int32_t* idx_out, int32_t* count_out, const lisa_linear_branch* lin, void* out,
+                              float* lse, void* ws, size_t ws_bytes, const lisa_stage_events* events,
+                              lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  const bool reuse = reuse_idx != nullptr || reuse_count != nullptr;
+  if (reuse && (reuse_idx == nullptr || reuse_count == nullptr)) return LISA_ERR_INVALID_ARG;
+  if ((idx_out == nullptr) != (count_out == nullptr)) return LISA_ERR_INVALID_ARG;
+  if (reuse && idx_out != nullptr) return LISA_ERR_INVALID_ARG;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || out == nullptr) return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  if (!reuse) {
+    LISA_TRY(check_idx_dim(desc));
+    if (P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr) return LISA_ERR_INVALID_ARG;
+    if (!aligned16(kproj_pool)) return LISA_ERR_INVALID_ARG;
+    if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
+  }
+  if (lin != nullptr && (lin->S == nullptr || lin->z == nullptr || lin->k_new == nullptr || lin->v_new == nullptr ||
+                         lin->gate_logit == nullptr))
+    return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  const int32_t* idx = reuse_idx;
+  const int32_t* count = reuse_count;
+  if (events) LISA_TRY(record(events->start, st));
+  if (!reuse) {
+    int32_t* di = idx_out ? idx_out : reinterpret_cast<int32_t*>(w + L.off_idx);
+    int32_t* dc = count_out ? count_out : reinterpret_cast<int32_t*>(w + L.off_count);
+    IndexParams p = index_params(*desc, L, ws);
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.P = P;
+    p.kproj = kproj_pool;
+    p.kproj_fp8 = kproj_dtype == LISA_KPROJ_FP8_E4M3;
+    p.kproj_scale = kproj_scale;
+    p.idx = di;
+    p.count = dc;
+    LISA_TRY(cuda_status(launch_index_select(p, false, st)));
+    idx = di;
+    count = dc;
+  }
+  if (events) LISA_TRY(record(events->after_index, st));
+  LISA_TRY(cuda_status(launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count), st)));
+  if (events) LISA_TRY(record(events->after_attn, st));
+  LISA_TRY(cuda_status(launch_merge(merge_params(*desc, L, ws, q, out, lse, lin), st)));
+  if (events) LISA_TRY(record(events->end, st));
+  return LISA_OK;
+}
+
+lisa_status lisa_check_device_error(void* ws, uint32_t* flags_out, lisa_stream_t stream) {
+  if (ws == nullptr) return LISA_ERR_WORKSPACE;
+  LISA_TRY(bind_device(ws));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess) return LISA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return LISA_ERR_CUDA;
+  if (word != 0 && cudaMemsetAsync(ws, 0, sizeof(word), st) != cudaSuccess) return LISA_ERR_CUDA;
+  if (flags_out) *flags_out = word;
+  return word != 0 ? LISA_ERR_DEVICE_CHECK : LISA_OK;
+}
+
+const char* lisa_status_string(lisa_status s) {
+  switch (s) {
+    case LISA_OK: return "ok";
+    case LISA_ERR_INVALID_ARG: return "invalid argument";
+    case LISA_ERR_UNSUPPORTED: return "unsupported shape";
+    case LISA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LISA_ERR_CUDA: return "CUDA error";
+    case LISA_ERR_DEVICE_CHECK: return "device-side range check failed";
+    case LISA_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

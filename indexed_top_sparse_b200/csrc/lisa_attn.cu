@@ -1,0 +1,396 @@
+// Attention stage of indexed sparse decode (sm_100a).
+//
+// What is computed (JSSA write-up, section "Как JSSA сохраняет порядок токенов", paragraphs on
+// decoding and on the specialised kernel): exact softmax attention of every query head over the
+// positions its KV head selected, using the original full-size bf16 keys and values read straight
+// from the paged cache -- no gathered copy -- with every head's own index set in one launch.  The
+// optional LISA linear branch and gate (LISA write-ups, "Архитектура LISA") are applied in the
+// merge kernel.
+//
+// Design on B200:
+//  * Split-KV: a CTA owns (partition of the index list, KV head, sequence).  Row addresses of its
+//    positions are resolved once through the page table into shared memory; then 64-position tiles
+//    of K and V rows (256 B each at d = 128) are copied with 16-byte cp.async into a 3-stage ring
+//    (XOR-swizzled rows), so ~64 KB per CTA are in flight while the previous tile is consumed.
+//  * The G query heads of one KV head are the n = 8 side of mma.m16n8k16 (bf16 in, fp32 accumulate):
+//    S^T = K Q^T with K rows from ldmatrix, then O^T += V^T P^T with V^T from ldmatrix.trans and P^T
+//    moved from the S^T accumulators by movmatrix.trans.  Tensor cores are used because the G-wide
+//    group makes this a real (if thin) contraction; the kernel stays bound by the row gathers.
+//  * Online softmax in base 2 per warp; warps merge in shared memory; partitions merge by
+//    log-sum-exp in the merge kernel, which also runs the linear branch and the gate.
+
+#include "lisa_common.cuh"
+#include "lisa_kernels.h"
+
+namespace lisa {
+
+namespace {
+
+#define kNegInf (__int_as_float(0xff800000u))
+
+template <int D>
+struct AttnGeom {
+  static constexpr int kRowBytes = D * 2;
+  static constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  static constexpr int kTileBytes = kAttnTile * kRowBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;  // K tile then V tile
+  static constexpr int kRowsPerPass = kAttnThreads / kChunks;
+  static constexpr size_t kSmem = (size_t)kAttnStages * kStageBytes + (size_t)kMaxSplitLen * 4;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
+  return (uint32_t)(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace
+
+size_t attn_smem_bytes(int d) { return d == 64 ? AttnGeom<64>::kSmem : AttnGeom<128>::kSmem; }
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnParams p) {
+  using Geo = AttnGeom<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint32_t* rows = reinterpret_cast<uint32_t*>(smem + kAttnStages * Geo::kStageBytes);
+
+  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g_ = lane >> 2, t_ = lane & 3;
+
+  int n = p.seq_lens[b];
+  if (n < 0 || n > p.max_seq_len) {
+    if (s == 0 && tid == 0) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
+    n = n < 0 ? 0 : p.max_seq_len;
+  }
+  const int limit = min(p.M, n);
+  int cnt = p.count[(size_t)b * p.Hkv + h];
+  if (cnt < 0 || cnt > limit) {
+    if (s == 0 && tid == 0) flag_error(p.err, LISA_DEVERR_COUNT);
+    cnt = cnt < 0 ? 0 : limit;
+  }
+  const int p0 = s * p.split_len;
+  const int len = max(0, min(cnt, p0 + p.split_len) - p0);
+
+  // Resolve the partition's positions to pool rows (row = (page * ps + slot) * Hkv + h).
+  const int32_t* idxp = p.idx + ((size_t)b * p.Hkv + h) * p.M + p0;
+  const int32_t* table = p.page_table + (size_t)b * p.max_pages;
+  for (int i = tid; i < len; i += kAttnThreads) {
+    int t = idxp[i];
+    if (t < 0 || t >= n) {
+      flag_error(p.err, LISA_DEVERR_INDEX);
+      t = 0;
+    }
+    int pg = table[t >> p.log2ps];
+    if (pg < 0 || pg >= p.num_pages) {
+      flag_error(p.err, LISA_DEVERR_PAGE_ID);
+      pg = 0;
+    }
+    rows[i] = ((uint32_t)pg * (uint32_t)p.ps + (uint32_t)(t & (p.ps - 1))) * (uint32_t)p.Hkv + (uint32_t)h;
+  }
+
+  // Q^T fragments (B operand, k = d, n = query head of the group); heads >= G are zero.
+  uint32_t qf[D / 16][2];
+  {
+    const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)h * G + (g_ < G ? g_ : 0)) * D;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      qf[kk][0] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_) : 0u;
+      qf[kk][1] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_ + 8) : 0u;
+    }
+  }
+  __syncthreads();
+
+  const int ntiles = (len + kAttnTile - 1) / kAttnTile;
+  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(p.k_pool);
+  const uint8_t* vbase = reinterpret_cast<const uint8_t*>(p.v_pool);
+  auto issue = [&](int tile, int stage) {
+    uint8_t* kdst = smem + stage * Geo::kStageBytes;
+    uint8_t* vdst = kdst + Geo::kTileBytes;
+    const int c = tid % Geo::kChunks;
+#pragma unroll
+    for (int r = tid / Geo::kChunks; r < kAttnTile; r += Geo::kRowsPerPass) {
+      const int li = tile * kAttnTile + r;
+      const bool valid = li < len;
+      const size_t off = (size_t)(valid ? rows[li] : 0u) * Geo::kRowBytes + (size_t)c * 16;
+      const uint32_t so = swz(r, c, Geo::kRowBytes);
+      cp_async_16(smem_u32(kdst + so), kbase + off, valid ? 16u : 0u);
+      cp_async_16(smem_u32(vdst + so), vbase + off, valid ? 16u : 0u);
+    }
+  };
+
+#pragma unroll
+  for (int st = 0; st < kAttnStages - 1; ++st) {
+    if (st < ntiles) issue(st, st);
+    cp_async_commit();
+  }
+
+  float m_run[2] = {kNegInf, kNegInf};  // per head 2t_, 2t_+1 (log2 units)
+  float l_run[2] = {0.f, 0.f};          // partial over this lane's rows
+  float o[D / 16][4];
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+  const int rbase = warp * 16;
+  for (int tile = 0; tile < ntiles; ++tile) {
+    const int nt = tile + kAttnStages - 1;
+    if (nt < ntiles) issue(nt, nt % kAttnStages);
+    cp_async_commit();
+    cp_async_wait<kAttnStages - 1>();
+    __syncthreads();
+
+    const uint8_t* ks = smem + (tile % kAttnStages) * Geo::kStageBytes;
+    const uint8_t* vs = ks + Geo::kTileBytes;
+
+    // S^T (16 positions x 8 heads) = K_tile(16 x D) . Q^T(D x 8)
+    float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int r = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int c = 2 * kk + (lane >> 4);
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(smem_u32(ks + swz(r, c, Geo::kRowBytes)), a0, a1, a2, a3);
+      mma_bf16_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+    }
+
+    // Online softmax (base 2).  c0,c1: position rbase+g_, heads 2t_,2t_+1; c2,c3: position +8.
+    const int pos0 = tile * kAttnTile + rbase + g_;
+    float x00 = sacc[0] * p.scale_log2, x01 = sacc[1] * p.scale_log2;
+    float x10 = sacc[2] * p.scale_log2, x11 = sacc[3] * p.scale_log2;
+    if (pos0 >= len) x00 = x01 = kNegInf;
+    if (pos0 + 8 >= len) x10 = x11 = kNegInf;
+    float mA = fmaxf(x00, x10), mB = fmaxf(x01, x11);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, off));
+      mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, off));
+    }
+    const float nA = fmaxf(m_run[0], mA), nB = fmaxf(m_run[1], mB);
+    const float alA = (nA == kNegInf) ? 1.f : exp2f(m_run[0] - nA);
+    const float alB = (nB == kNegInf) ? 1.f : exp2f(m_run[1] - nB);
+    const float pA0 = (nA == kNegInf) ? 0.f : exp2f(x00 - nA);
+    const float pA1 = (nA == kNegInf) ? 0.f : exp2f(x10 - nA);
+    const float pB0 = (nB == kNegInf) ? 0.f : exp2f(x01 - nB);
+    const float pB1 = (nB == kNegInf) ? 0.f : exp2f(x11 - nB);
+    l_run[0] = l_run[0] * alA + pA0 + pA1;
+    l_run[1] = l_run[1] * alB + pB0 + pB1;
+    m_run[0] = nA;
+    m_run[1] = nB;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      o[mt][0] *= alA;
+      o[mt][1] *= alB;
+      o[mt][2] *= alA;
+      o[mt][3] *= alB;
+    }
+    // P^T (16 positions x 8 heads) in bf16 -> B fragments of the PV product via an 8x8 transpose.
+    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(pA0, pB0));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(pA1, pB1));
+
+    // O^T (D x 8) += V^T(D x 16 positions) . P^T(16 x 8)
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const int r = rbase + (lane & 7) + ((lane >> 4) & 1) * 8;
+      const int c = 2 * mt + ((lane >> 3) & 1);
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4_trans(smem_u32(vs + swz(r, c, Geo::kRowBytes)), a0, a1, a2, a3);
+      mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+    }
+    __syncthreads();  // the stage is refilled by a later iteration
+  }
+  cp_async_wait<0>();
+
+  // Reduce the lane-partial sums over the 8 row groups.
+#pragma unroll
+  for (int off = 4; off < 32; off <<= 1) {
+    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+  }
+  __syncthreads();
+  // Per-warp results to shared memory: obuf[warp][head][D], wm/wl[warp][head].
+  float* obuf = reinterpret_cast<float*>(smem);
+  float* wm = obuf + 4 * kMaxG * D;
+  float* wl = wm + 4 * kMaxG;
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) {
+    const int d0 = 16 * mt + g_;
+    obuf[(warp * kMaxG + 2 * t_) * D + d0] = o[mt][0];
+    obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0] = o[mt][1];
+    obuf[(warp * kMaxG + 2 * t_) * D + d0 + 8] = o[mt][2];
+    obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0 + 8] = o[mt][3];
+  }
+  if (g_ == 0) {
+    wm[warp * kMaxG + 2 * t_] = m_run[0];
+    wm[warp * kMaxG + 2 * t_ + 1] = m_run[1];
+    wl[warp * kMaxG + 2 * t_] = l_run[0];
+    wl[warp * kMaxG + 2 * t_ + 1] = l_run[1];
+  }
+  __syncthreads();
+  const size_t part = ((size_t)b * p.Hkv + h) * p.splits + s;
+  float* op = p.o_part + part * G * D;
+  for (int e = tid; e < G * D; e += kAttnThreads) {
+    const int gg = e / D, dd = e - gg * D;
+    float mx = kNegInf;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + gg]);
+    float acc = 0.f;
+    if (mx != kNegInf) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = wm[w * kMaxG + gg];
+        if (mw != kNegInf) acc += obuf[(w * kMaxG + gg) * D + dd] * exp2f(mw - mx);
+      }
+    }
+    op[e] = acc;
+  }
+  if (tid < G) {
+    float mx = kNegInf;
+    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + tid]);
+    float l = 0.f;
+    if (mx != kNegInf) {
+      for (int w = 0; w < 4; ++w) {
+        const float mw = wm[w * kMaxG + tid];
+        if (mw != kNegInf) l += wl[w * kMaxG + tid] * exp2f(mw - mx);
+      }
+    }
+    p.ml_part[(part * G + tid) * 2 + 0] = mx;
+    p.ml_part[(part * G + tid) * 2 + 1] = l;
+  }
+}
+
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// Merge the partitions of one (b, KV head) for its G query heads; optional linear branch + gate.
+// One CTA per (KV head, sequence); thread e owns output column e.
+template <int D>
+__global__ void __launch_bounds__(128) lisa_merge_kernel(MergeParams p) {
+  __shared__ float fk[D];
+  __shared__ float fq[kMaxG][D];
+  __shared__ float zn[D];
+  __shared__ float den[kMaxG];
+  __shared__ float wsplit[kMaxG][64];
+  __shared__ float mstar[kMaxG], lstar[kMaxG];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const float* mlp = p.ml_part + bh * p.splits * G * 2;
+  const float* op = p.o_part + bh * p.splits * G * D;
+
+  // Partition weights, in chunks of 64 partitions.
+  float acc[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  if (tid < G) {
+    float mx = kNegInf;
+    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, mlp[(s * G + tid) * 2]);
+    float l = 0.f;
+    if (mx != kNegInf)
+      for (int s = 0; s < p.splits; ++s) {
+        const float ms = mlp[(s * G + tid) * 2];
+        if (ms != kNegInf) l += mlp[(s * G + tid) * 2 + 1] * exp2f(ms - mx);
+      }
+    mstar[tid] = mx;
+    lstar[tid] = l;
+  }
+  for (int s0 = 0; s0 < p.splits; s0 += 64) {
+    __syncthreads();
+    for (int e = tid; e < G * 64; e += blockDim.x) {
+      const int g = e / 64, s = s0 + (e - g * 64);
+      float w = 0.f;
+      if (s < p.splits) {
+        const float ms = mlp[(s * G + g) * 2];
+        if (ms != kNegInf && mstar[g] != kNegInf) w = exp2f(ms - mstar[g]);
+      }
+      wsplit[g][e - g * 64] = w;
+    }
+    __syncthreads();
+    if (tid < D) {
+      const int s1 = min(p.splits, s0 + 64);
+      for (int s = s0; s < s1; ++s)
+        for (int g = 0; g < G; ++g) acc[g] += wsplit[g][s - s0] * op[((size_t)s * G + g) * D + tid];
+    }
+  }
+  float sparse[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) sparse[g] = (g < G && lstar[g] > 0.f) ? acc[g] / lstar[g] : 0.f;
+  if (p.lse != nullptr && tid < G) {
+    const float l = lstar[tid];
+    p.lse[(size_t)b * p.Hq + (size_t)h * G + tid] =
+        l > 0.f ? (mstar[tid] + log2f(l)) * 0.69314718055994530942f : kNegInf;
+  }
+
+  float outv[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) outv[g] = sparse[g];
+  if (p.S != nullptr) {
+    // Linear branch: S += phi(k) v^T, z += phi(k); lin_g = phi(q_g)^T S / (phi(q_g) . z).
+    if (tid < D) {
+      const float f = phi_elu1(__bfloat162float(p.k_new[bh * D + tid]));
+      fk[tid] = f;
+      zn[tid] = p.z[bh * D + tid] + f;
+      for (int g = 0; g < G; ++g)
+        fq[g][tid] = phi_elu1(__bfloat162float(p.q[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid]));
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += blockDim.x >> 5) {
+      float a = 0.f;
+      for (int c = lane; c < D; c += 32) a = fmaf(fq[g][c], zn[c], a);
+      a = warp_sum(a);
+      if (lane == 0) den[g] = a;
+    }
+    if (tid < D) p.z[bh * D + tid] = zn[tid];
+    __syncthreads();
+    if (tid < D) {
+      float lin[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) lin[g] = 0.f;
+      const float ve = __bfloat162float(p.v_new[bh * D + tid]);
+      float* Sbh = p.S + bh * D * D;
+      for (int c = 0; c < D; ++c) {
+        const float sn = fmaf(fk[c], ve, Sbh[(size_t)c * D + tid]);
+        Sbh[(size_t)c * D + tid] = sn;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) lin[g] = fmaf(fq[g][c], sn, lin[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) {
+        if (g < G) {
+          const float sg = 1.f / (1.f + expf(-p.gate[(size_t)h * G + g]));
+          outv[g] = sg * sparse[g] + (1.f - sg) * (lin[g] / den[g]);
+        }
+      }
+    }
+  }
+  if (tid < D) {
+    for (int g = 0; g < G; ++g)
+      p.out[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid] = __float2bfloat16_rn(outv[g]);
+  }
+}
+
+cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream) {
+  dim3 grid(p.splits, p.Hkv, p.B);
+  if (p.d == 64) {
+    auto k = lisa_sparse_attn_kernel<64>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<64>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kAttnThreads, AttnGeom<64>::kSmem, stream>>>(p);
+  } else {
+    auto k = lisa_sparse_attn_kernel<128>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<128>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kAttnThreads, AttnGeom<128>::kSmem, stream>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
+  dim3 grid(p.Hkv, p.B);
+  if (p.d == 64)
+    lisa_merge_kernel<64><<<grid, 128, 0, stream>>>(p);
+  else
+    lisa_merge_kernel<128><<<grid, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace lisa

@@ -1,0 +1,67 @@
+// Internal interface between the C ABI layer and the kernels (not installed, not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lisa {
+
+constexpr int kScoreChunk = 4096;  // positions per CTA of the score-only kernel
+
+struct IndexParams {
+  int B, Hq, Hkv, d, r, M, ps, log2ps, max_pages, max_seq_len, num_pages;
+  int chunk_max;  // positions per CTA of a select cluster, at most (multiple of ps)
+  bool kproj_fp8;
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  const __nv_bfloat16* q;
+  const float* P;
+  const void* kproj;
+  const float* kproj_scale;
+  float* scores;  // written by the score kernel, read by the select-from-scores kernel
+  int32_t* idx;
+  int32_t* count;
+  uint32_t* err;
+};
+
+struct AttnParams {
+  int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
+  int splits, split_len;
+  float scale_log2;  // softmax scale * log2(e)
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_pool;
+  const __nv_bfloat16* v_pool;
+  const int32_t* idx;
+  const int32_t* count;
+  float* o_part;   // [B][Hkv][splits][G][d], unnormalised, relative to the partition max
+  float* ml_part;  // [B][Hkv][splits][G][2]: (max in log2 units, sum of 2^(x - max))
+  uint32_t* err;
+};
+
+struct MergeParams {
+  int B, Hq, Hkv, d, splits;
+  const float* o_part;
+  const float* ml_part;
+  const __nv_bfloat16* q;
+  __nv_bfloat16* out;
+  float* lse;  // nullable
+  // linear branch (all null when absent)
+  float* S;
+  float* z;
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  const float* gate;
+};
+
+size_t select_smem_bytes(int chunk_max, int ps);
+size_t attn_smem_bytes(int d);
+cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
+cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
+cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
+
+}  // namespace lisa

@@ -1,0 +1,123 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry point, and the host-side
+argument checks return the documented status codes (no compute calls -- these run without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import indexed_top_sparse_b200 as L
+from indexed_top_sparse_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "lisa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lisa_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    declared = _declared_functions()
+    assert len(declared) >= 9
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(B.EXPORTED) == declared
+
+
+def _desc(**kw):
+    base = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, idx_dim=32, budget_m=256, page_size=64,
+                max_pages_per_seq=16, max_seq_len=1024, num_pages=32)
+    base.update(kw)
+    d = L.make_desc(**base)
+    # non-null placeholders for the device tables: validation does not dereference them
+    d.seq_lens = 0x1000
+    d.page_table = 0x2000
+    return d
+
+
+def test_workspace_size_and_splits():
+    d = _desc()
+    ws = L.lisa_workspace_size(d)
+    splits = L.lisa_num_splits(d)
+    assert splits >= 1 and ws > 256
+    assert ws % 256 == 0
+    # partitions cover the budget with at most 1024 positions each
+    assert splits * 1024 >= 256
+    big = _desc(budget_m=16384, batch=1, num_kv_heads=1, num_q_heads=8, max_seq_len=131072, max_pages_per_seq=2048,
+                num_pages=2048)
+    assert L.lisa_num_splits(big) >= 16
+
+
+@pytest.mark.parametrize(
+    "kw,status",
+    [
+        (dict(head_dim=96), 2),
+        (dict(idx_dim=24), 2),
+        (dict(num_q_heads=72, num_kv_heads=8), 2),  # G = 9 > 8
+        (dict(num_q_heads=7), 1),  # not a multiple of Hkv
+        (dict(page_size=48, max_pages_per_seq=32), 2),
+        (dict(page_size=8, max_pages_per_seq=128), 2),
+        (dict(budget_m=0), 1),
+        (dict(budget_m=16385), 2),
+        (dict(max_seq_len=262145, max_pages_per_seq=5000), 2),
+        (dict(max_pages_per_seq=15), 1),  # 15 * 64 < 1024
+        (dict(num_pages=0), 1),
+        (dict(batch=-1), 1),
+    ],
+)
+def test_host_argument_checks(kw, status):
+    d = _desc(**kw)
+    st = B._lib.lisa_index_topm(ctypes.byref(d), 0x1000, 0x1000, 0x1000, 1, 0x1000, 0x1000, 0x1000, 0x100, 1 << 30, None)
+    assert st == status, B.STATUS_NAMES.get(st)
+    if "idx_dim" not in kw:  # r is checked by the index entry points only
+        assert L.lisa_workspace_size(d) == 0
+
+
+def test_null_and_workspace_checks():
+    d = _desc()
+    need = L.lisa_workspace_size(d)
+    lib = B._lib
+    A = 0x1000  # aligned placeholder pointer: these calls stop at the host checks
+    # null desc
+    assert lib.lisa_sparse_decode_attn(None, A, A, A, A, A, A, None, 0x100, need, None) == 1
+    # null required pointer
+    assert lib.lisa_sparse_decode_attn(ctypes.byref(d), None, A, A, A, A, A, None, 0x100, need, None) == 1
+    # misaligned pools (cp.async / 16-byte loads need 16-byte alignment)
+    assert lib.lisa_sparse_decode_attn(ctypes.byref(d), A, A + 8, A, A, A, A, None, 0x100, need, None) == 1
+    assert lib.lisa_index_topm(ctypes.byref(d), A, A, A + 4, 1, A, A, A, 0x100, need, None) == 1
+    # workspace: null, misaligned, too small
+    assert lib.lisa_sparse_decode_attn(ctypes.byref(d), A, A, A, A, A, A, None, None, need, None) == 3
+    assert lib.lisa_sparse_decode_attn(ctypes.byref(d), A, A, A, A, A, A, None, 0x108, need, None) == 3
+    assert lib.lisa_sparse_decode_attn(ctypes.byref(d), A, A, A, A, A, A, None, 0x100, need - 1, None) == 3
+    # reuse pointers must come in pairs and exclude idx_out
+    args = [ctypes.byref(d), A, A, A, 1, A, A, A]
+    assert lib.lisa_fused_decode(*args, A, None, None, None, None, A, None, 0x100, need, None, None) == 1
+    assert lib.lisa_fused_decode(*args, A, A, A, A, None, A, None, 0x100, need, None, None) == 1
+    assert lib.lisa_fused_decode(*args, None, None, A, None, None, A, None, 0x100, need, None, None) == 1
+    # bad kproj dtype
+    assert lib.lisa_index_score(ctypes.byref(d), A, A, A, 7, A, A, 0x100, need, None) == 1
+
+
+def test_empty_batch_is_a_no_op():
+    d = _desc(batch=0)
+    d.seq_lens = None
+    d.page_table = None
+    assert B._lib.lisa_index_topm(ctypes.byref(d), None, None, None, 1, None, None, None, None, 0, None) == 0
+    assert B._lib.lisa_fused_decode(ctypes.byref(d), *([None] * 3), 1, *([None] * 11), 0, None, None) == 0
+
+
+def test_status_strings():
+    for s in range(7):
+        assert L.lisa_status_string(s) != "unknown status"
+    assert L.lisa_status_string(99) == "unknown status"
+
+
+def test_binding_refuses_non_contiguous():
+    x = torch.zeros(4, 4)[:, ::2]
+    with pytest.raises(ValueError):
+        B._ptr(x)

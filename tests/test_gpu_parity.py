@@ -1,0 +1,349 @@
+"""GPU parity of the C-ABI entry points against the fp64 oracle, on seeded inputs.
+
+Small cases are checked element by element over every (sequence, KV head); the full-size
+workloads (128K paged, ragged 64-sequence batch, layered hybrid) are run in the launch
+configuration the benchmark times and checked on sampled sequences.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import indexed_top_sparse_b200 as L
+from oracle import lisa_oracle as O
+from tests.parity import check_index_sets, check_outputs
+from workloads import config1, config2, config3, config4, config5, make_problem
+from workloads import run as R
+from workloads.host_view import host_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def all_pairs(prob):
+    return [(b, h) for b in range(prob.B) for h in range(prob.Hkv)]
+
+
+def small(dev, **kw):
+    args = dict(name="case", B=2, Hq=8, Hkv=2, d=128, r=32, M=256, seq_lens=[5000, 3001], page_size=64, paged=False,
+                kproj_fp8=True, plant=("cosine", 0.01), seed=77)
+    args.update(kw)
+    return make_problem(device=dev, **args)
+
+
+CASES = {
+    "c1": lambda dev: config1(device=dev),
+    "fp8_r32_contig": lambda dev: small(dev),
+    "fp8_r16_paged_d64": lambda dev: small(dev, B=3, Hq=6, Hkv=3, d=64, r=16, M=100, seq_lens=[777, 4096, 9000],
+                                            page_size=16, paged=True, seed=78),
+    "fp32_r32_paged_g4": lambda dev: small(dev, B=2, Hq=4, Hkv=1, r=32, M=64, seq_lens=[1500, 64], page_size=128,
+                                           paged=True, kproj_fp8=False, seed=79),
+    "g8_ps1024": lambda dev: small(dev, B=2, Hq=16, Hkv=2, M=512, seq_lens=[20000, 2500], page_size=1024,
+                                   paged=True, seed=80),
+    "g1": lambda dev: small(dev, B=2, Hq=3, Hkv=3, M=300, seq_lens=[4000, 301], paged=True, seed=81),
+    "c2_full": lambda dev: config2(device=dev),
+}
+
+
+# ---------------------------------------------------------------------------------------------
+# Stage by stage
+# ---------------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_index_score_parity(cuda_device, case):
+    prob = CASES[case](cuda_device)
+    ws = R.workspace(prob)
+    scores = f64(R.index_scores(prob, ws))
+    assert L.lisa_check_device_error(ws) == 0
+    inp = host_inputs(prob)
+    for b, h in all_pairs(prob):
+        n = int(prob.seq_lens[b])
+        ref = O.head_scores(inp, b, h)
+        got = scores[b, h, :n]
+        tol = 1e-5 * max(np.max(np.abs(ref)), 1e-30)
+        assert np.max(np.abs(got - ref)) <= tol, (case, b, h, np.max(np.abs(got - ref)), tol)
+        assert np.all(np.isnan(scores[b, h, n:])), "entries past n_b must not be written"
+
+
+def _select_desc(B, Hkv, M, max_len, dev):
+    ps = 64
+    mp = -(-max_len // ps)
+    table = torch.arange(B * mp, dtype=torch.int32, device=dev).view(B, mp)
+    return table, dict(batch=B, num_q_heads=Hkv, num_kv_heads=Hkv, head_dim=128, idx_dim=32, budget_m=M,
+                       page_size=ps, max_pages_per_seq=mp, max_seq_len=max_len, num_pages=B * mp)
+
+
+SELECT_CASES = [
+    # (seq_lens, Hkv, M, mode)
+    ([1, 5], 2, 5, "normal"),
+    ([48, 100], 1, 64, "normal"),
+    ([2047, 2048, 2049], 2, 2048, "normal"),
+    ([131072], 2, 2048, "normal"),
+    ([5000, 777], 3, 1, "normal"),
+    ([70000], 1, 16384, "normal"),
+    ([9000, 4100], 2, 300, "ties"),
+    ([6000], 2, 1000, "all_equal"),
+    ([30000, 12345], 2, 2048, "coarse"),
+]
+
+
+@pytest.mark.parametrize("lens,Hkv,M,mode", SELECT_CASES)
+def test_topm_select_bit_exact(cuda_device, lens, Hkv, M, mode):
+    """Scores chosen here (fp32 values), selection by the library vs the oracle: identical index sets."""
+    rng = np.random.default_rng(sum(lens) + M)
+    B, max_len = len(lens), max(lens)
+    s = np.full((B, Hkv, max_len), np.nan, dtype=np.float32)  # never read past n_b
+    for b, n in enumerate(lens):
+        for h in range(Hkv):
+            v = rng.standard_normal(n).astype(np.float32) * 3
+            if mode == "ties" and n > M:
+                thr = np.sort(v)[::-1][M - 1]
+                v[rng.choice(n, 40, replace=False)] = thr  # many exact ties at the M-th score
+            elif mode == "all_equal":
+                v[:] = 1.25
+            elif mode == "coarse":
+                v = np.round(v, 1).astype(np.float32)
+                v[rng.choice(n, 5, replace=False)] = -0.0
+            s[b, h, :n] = v
+    table, kw = _select_desc(B, Hkv, M, max_len, cuda_device)
+    seq = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
+    desc = L.make_desc(seq_lens=seq, page_table=table, **kw)
+    ws = L.alloc_workspace(desc, cuda_device)
+    scores = torch.from_numpy(s).to(cuda_device)
+    idx = torch.full((B, Hkv, M), -7, dtype=torch.int32, device=cuda_device)
+    count = torch.full((B, Hkv), -7, dtype=torch.int32, device=cuda_device)
+    L.lisa_topm_select(desc, scores, idx, count, ws)
+    idx, count = idx.cpu().numpy(), count.cpu().numpy()
+    assert L.lisa_check_device_error(ws) == 0
+    for b, n in enumerate(lens):
+        for h in range(Hkv):
+            want = O.select_top_m(s[b, h, :n].astype(np.float64), M)
+            m = len(want)
+            assert count[b, h] == m
+            assert np.array_equal(idx[b, h, :m], want), (b, h, mode)
+            assert np.all(idx[b, h, m:] == -1)
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_index_topm_parity(cuda_device, case):
+    prob = CASES[case](cuda_device)
+    ws = R.workspace(prob)
+    idx, count = R.index_topm(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    inp = host_inputs(prob)
+    ref = O.decode_step(inp)
+    same = check_index_sets(idx.cpu().numpy(), count.cpu().numpy(), ref, inp["seq_lens"], prob.M, all_pairs(prob))
+    assert len(same) >= 0.9 * len(all_pairs(prob))
+    if prob.planted is not None and case == "c1":
+        assert set(prob.planted[0][0].tolist()) <= set(idx[0, 0].tolist())
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_attention_parity_given_oracle_index(cuda_device, case):
+    """Index sets chosen by the oracle, attention by the library."""
+    prob = CASES[case](cuda_device)
+    inp = host_inputs(prob)
+    ref = O.decode_step(inp)
+    idx = np.full((prob.B, prob.Hkv, prob.M), -1, dtype=np.int32)
+    count = np.zeros((prob.B, prob.Hkv), dtype=np.int32)
+    for b, h in all_pairs(prob):
+        sel = ref["idx"][b][h]
+        idx[b, h, : len(sel)] = sel
+        count[b, h] = len(sel)
+    ws = R.workspace(prob)
+    out, lse = R.attention(prob, torch.from_numpy(idx).to(cuda_device), torch.from_numpy(count).to(cuda_device), ws)
+    assert L.lisa_check_device_error(ws) == 0
+    check_outputs(f64(out), ref["out"], all_pairs(prob), prob.G)
+    assert np.allclose(f64(lse), ref["lse"], rtol=1e-5, atol=1e-4)
+
+
+# ---------------------------------------------------------------------------------------------
+# Whole path
+# ---------------------------------------------------------------------------------------------
+
+
+def _fused_vs_oracle(prob, seqs=None, min_identical=0.9):
+    ws = R.workspace(prob)
+    res = R.fused(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    seqs = list(range(prob.B)) if seqs is None else list(seqs)
+    inp = host_inputs(prob, seqs=seqs)
+    ref = O.decode_step(inp)
+    pairs = [(i, h) for i in range(len(seqs)) for h in range(prob.Hkv)]
+    sel = torch.tensor(seqs, device=prob.device)
+    gi = res["idx"][sel].cpu().numpy()
+    gc = res["count"][sel].cpu().numpy()
+    same = check_index_sets(gi, gc, ref, inp["seq_lens"], prob.M, pairs)
+    assert len(same) >= min_identical * len(pairs), (len(same), len(pairs))
+    worst = check_outputs(f64(res["out"][sel]), ref["out"], same, prob.G)
+    lse = f64(res["lse"][sel])
+    for i, h in same:
+        rows = slice(h * prob.G, (h + 1) * prob.G)
+        assert np.allclose(lse[i, rows], ref["lse"][i, rows], rtol=1e-5, atol=1e-4)
+    return worst
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_fused_decode_parity(cuda_device, case):
+    _fused_vs_oracle(CASES[case](cuda_device))
+
+
+@pytest.mark.parametrize("n", [1, 48, 2047, 2048, 2049, 4160])
+def test_context_around_budget(cuda_device, n):
+    prob = small(cuda_device, B=2, M=2048, seq_lens=[n, max(1, n // 3)], paged=True, seed=90 + n)
+    _fused_vs_oracle(prob)
+
+
+def test_budget_one(cuda_device):
+    _fused_vs_oracle(small(cuda_device, M=1, seq_lens=[3000, 17], seed=91))
+
+
+def test_fused_is_deterministic(cuda_device):
+    prob = small(cuda_device, seed=92)
+    ws = R.workspace(prob)
+    a = R.fused(prob, ws)
+    b = R.fused(prob, ws)
+    assert torch.equal(a["idx"], b["idx"]) and torch.equal(a["out"], b["out"]) and torch.equal(a["lse"], b["lse"])
+
+
+def test_empty_sequence(cuda_device):
+    prob = small(cuda_device, seq_lens=[3000, 1], seed=93)
+    prob.seq_lens[1] = 0
+    ws = R.workspace(prob)
+    res = R.fused(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    assert int(res["count"][1, 0]) == 0 and int(res["count"][1, 1]) == 0
+    assert torch.all(res["idx"][1] == -1)
+    assert torch.all(res["out"][1].float() == 0)
+    assert torch.all(torch.isneginf(res["lse"][1]))
+
+
+def test_device_range_checks_flag_without_faulting(cuda_device):
+    prob = small(cuda_device, seq_lens=[3000, 1000], paged=True, seed=94)
+    ws = R.workspace(prob)
+    # a page id past the pool
+    bad = prob.page_table.clone()
+    prob.page_table[0, 3] = prob.num_pages + 5
+    desc = R.desc_of(prob)
+    R.fused(prob, ws, desc=desc)
+    assert L.lisa_check_device_error(ws) & L.DEVERR_PAGE_ID
+    assert L.lisa_check_device_error(ws) == 0  # cleared by the read
+    prob.page_table.copy_(bad)
+    # an index past n_b and a count past min(M, n_b)
+    idx = torch.zeros(prob.B, prob.Hkv, prob.M, dtype=torch.int32, device=cuda_device)
+    idx[0, 0, 0] = 5000
+    count = torch.full((prob.B, prob.Hkv), 3, dtype=torch.int32, device=cuda_device)
+    count[1, 1] = prob.M + 1
+    R.attention(prob, idx, count, ws)
+    flags = L.lisa_check_device_error(ws)
+    assert flags & L.DEVERR_INDEX and flags & L.DEVERR_COUNT
+    # a sequence length past max_seq_len
+    prob.seq_lens[1] = prob.max_seq_len + 1
+    R.index_topm(prob, ws)
+    assert L.lisa_check_device_error(ws) & L.DEVERR_SEQ_LEN
+
+
+# ---------------------------------------------------------------------------------------------
+# Hybrid layers: linear branch, gate and cross-layer reuse
+# ---------------------------------------------------------------------------------------------
+
+
+def _run_layers(lp, dev):
+    outs = []
+    state = [p.lin.clone() for p in lp.layers]
+    last = None
+    for layer, prob in enumerate(lp.layers):
+        ws = R.workspace(prob)
+        if layer in lp.full_layers:
+            res = R.fused(prob, ws, lin=state[layer])
+            last = (res["idx"], res["count"])
+        else:
+            res = R.fused(prob, ws, reuse=last, lin=state[layer])
+            res["idx"], res["count"] = last
+        assert L.lisa_check_device_error(ws) == 0
+        outs.append(res)
+    return outs, state
+
+
+def test_layered_hybrid_parity(cuda_device):
+    lp = config5(device=cuda_device, layers=8, B=2, n=8192, M=1024)
+    outs, state = _run_layers(lp, cuda_device)
+    inps = [host_inputs(p) for p in lp.layers]
+    refs = O.layered_decode(inps, lp.full_layers)
+    prob0 = lp.layers[0]
+    pairs = all_pairs(prob0)
+    for layer in range(8):
+        src = lp.source_layer(layer)
+        gi = outs[layer]["idx"].cpu().numpy()
+        gc = outs[layer]["count"].cpu().numpy()
+        if layer in lp.full_layers:
+            same = check_index_sets(gi, gc, refs[layer], inps[layer]["seq_lens"], prob0.M, pairs)
+        else:
+            assert np.array_equal(gi, outs[src]["idx"].cpu().numpy())  # reused verbatim
+            same = [pr for pr in pairs if np.array_equal(gi[pr[0], pr[1], : gc[pr]], refs[src]["idx"][pr[0]][pr[1]])]
+        check_outputs(f64(outs[layer]["out"]), refs[layer]["out"], same, prob0.G)
+        # the linear state is updated in place (fp32 on the device vs fp64)
+        assert np.allclose(state[layer].S.cpu().numpy(), refs[layer]["S"], rtol=1e-5, atol=1e-3)
+        assert np.allclose(state[layer].z.cpu().numpy(), refs[layer]["z"], rtol=1e-6, atol=1e-4)
+
+
+def test_gate_extremes_on_device(cuda_device):
+    lp = config5(device=cuda_device, layers=1, full_layers=(0,), B=1, Hq=8, Hkv=2, n=2000, M=256)
+    prob = lp.layers[0]
+    for g, which in ((60.0, "sparse"), (-60.0, "linear")):
+        lin = prob.lin.clone()
+        lin.gate.fill_(g)
+        ws = R.workspace(prob)
+        res = R.fused(prob, ws, lin=lin)
+        inp = host_inputs(prob, lin=lin)
+        ref = O.decode_step(inp)
+        check_outputs(f64(res["out"]), ref["out"], all_pairs(prob), prob.G)
+        if which == "sparse":
+            plain = R.fused(prob, R.workspace(prob))
+            assert torch.allclose(res["out"].float(), plain["out"].float(), rtol=0, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------------------------
+# Full-size workloads, sampled
+# ---------------------------------------------------------------------------------------------
+
+
+def test_full_size_128k_paged_sampled(cuda_device):
+    prob = config3(device=cuda_device)
+    _fused_vs_oracle(prob, seqs=[0, 9, 15])
+    del prob
+    torch.cuda.empty_cache()
+
+
+def test_full_size_ragged_batch_sampled(cuda_device):
+    prob = config4(device=cuda_device)
+    lens = prob.seq_lens.tolist()
+    seqs = sorted({int(np.argmin(lens)), int(np.argmax(lens)), 17})
+    _fused_vs_oracle(prob, seqs=seqs)
+    del prob
+    torch.cuda.empty_cache()
+
+
+def test_full_size_hybrid_sampled(cuda_device):
+    lp = config5(device=cuda_device)
+    outs, state = _run_layers(lp, cuda_device)
+    seqs = [0, 5]
+    inps = [host_inputs(p, seqs=seqs, lin=p.lin) for p in lp.layers]
+    refs = O.layered_decode(inps, lp.full_layers)
+    sel = torch.tensor(seqs, device=cuda_device)
+    prob0 = lp.layers[0]
+    pairs = [(i, h) for i in range(len(seqs)) for h in range(prob0.Hkv)]
+    for layer in range(len(lp.layers)):
+        src = lp.source_layer(layer)
+        gi = outs[src]["idx"][sel].cpu().numpy()
+        gc = outs[src]["count"][sel].cpu().numpy()
+        same = check_index_sets(gi, gc, refs[src], inps[src]["seq_lens"], prob0.M, pairs)
+        check_outputs(f64(outs[layer]["out"][sel]), refs[layer]["out"], same, prob0.G)
+    del lp, outs, state
+    torch.cuda.empty_cache()

@@ -1,0 +1,85 @@
+"""Drive the library's C entry points on a DecodeProblem (device tensors in, device tensors out).
+
+Marshalling only: descriptors, output buffers and workspace come from here;
+every step of the decode path runs inside the library.
+"""
+
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+import indexed_top_sparse_b200 as L
+
+from .synth import DecodeProblem
+
+
+def desc_of(prob: DecodeProblem) -> L.DecodeDesc:
+    return L.make_desc(
+        batch=prob.B, num_q_heads=prob.Hq, num_kv_heads=prob.Hkv, head_dim=prob.d, idx_dim=prob.r,
+        budget_m=prob.M, page_size=prob.page_size, max_pages_per_seq=prob.max_pages,
+        max_seq_len=prob.max_seq_len, num_pages=prob.num_pages, seq_lens=prob.seq_lens,
+        page_table=prob.page_table, softmax_scale=prob.softmax_scale,
+    )
+
+
+def kproj_dtype(prob: DecodeProblem) -> int:
+    return L.KPROJ_FP8_E4M3 if prob.kproj_fp8 else L.KPROJ_FP32
+
+
+def workspace(prob: DecodeProblem, desc=None) -> torch.Tensor:
+    return L.alloc_workspace(desc or desc_of(prob), prob.device)
+
+
+def index_scores(prob: DecodeProblem, ws: torch.Tensor, desc=None) -> torch.Tensor:
+    desc = desc or desc_of(prob)
+    scores = torch.full((prob.B, prob.Hkv, prob.max_seq_len), float("nan"), dtype=torch.float32, device=prob.device)
+    L.lisa_index_score(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), prob.kproj_scale.to(prob.device), scores, ws)
+    return scores
+
+
+def topm_from_scores(prob: DecodeProblem, scores: torch.Tensor, ws: torch.Tensor, desc=None):
+    desc = desc or desc_of(prob)
+    idx = torch.full((prob.B, prob.Hkv, prob.M), -7, dtype=torch.int32, device=prob.device)
+    count = torch.full((prob.B, prob.Hkv), -7, dtype=torch.int32, device=prob.device)
+    L.lisa_topm_select(desc, scores, idx, count, ws)
+    return idx, count
+
+
+def index_topm(prob: DecodeProblem, ws: torch.Tensor, desc=None):
+    desc = desc or desc_of(prob)
+    idx = torch.full((prob.B, prob.Hkv, prob.M), -7, dtype=torch.int32, device=prob.device)
+    count = torch.full((prob.B, prob.Hkv), -7, dtype=torch.int32, device=prob.device)
+    L.lisa_index_topm(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), prob.kproj_scale.to(prob.device), idx,
+                      count, ws)
+    return idx, count
+
+
+def attention(prob: DecodeProblem, idx: torch.Tensor, count: torch.Tensor, ws: torch.Tensor, desc=None):
+    desc = desc or desc_of(prob)
+    out = torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=prob.device)
+    lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=prob.device)
+    L.lisa_sparse_decode_attn(desc, prob.q, prob.k_pool, prob.v_pool, idx, count, out, lse, ws)
+    return out, lse
+
+
+def fused(prob: DecodeProblem, ws: torch.Tensor, desc=None, reuse: Optional[tuple] = None, return_idx=True,
+          lin=None, events=None, stream=None, out=None, lse=None):
+    """One call of lisa_fused_decode.  lin: a workloads LinearBranchInputs (state updated in place)."""
+    desc = desc or desc_of(prob)
+    dev = prob.device
+    out = out if out is not None else torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=dev)
+    lse = lse if lse is not None else torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=dev)
+    idx = count = None
+    if return_idx and reuse is None:
+        idx = torch.full((prob.B, prob.Hkv, prob.M), -7, dtype=torch.int32, device=dev)
+        count = torch.full((prob.B, prob.Hkv), -7, dtype=torch.int32, device=dev)
+    lb = None
+    if lin is not None:
+        lb = L.linear_branch(lin.S, lin.z, lin.k_new, lin.v_new, lin.gate)
+    ridx, rcount = (None, None) if reuse is None else reuse
+    scale = prob.kproj_scale.to(dev) if prob.kproj is not None else None
+    L.lisa_fused_decode(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), scale, prob.k_pool, prob.v_pool, ridx,
+                        rcount, idx, count, lb, out, lse, ws, events=events, stream=stream)
+    return {"out": out, "lse": lse, "idx": idx, "count": count}
