@@ -36,6 +36,8 @@
  *   - Values that can only be checked on the device (sequence lengths, page ids, indices, counts) are
  *     checked by the kernels: an out-of-range value is clamped to a safe one, the computation goes on,
  *     and a sticky bit is set in the workspace error word, read by lisa_check_device_error.
+ *   - Alignment: kproj_pool 32 bytes, k_pool/v_pool 16 bytes, q and scores 4 bytes (LISA_ERR_INVALID_ARG
+ *     otherwise); every allocation from cudaMalloc or torch meets this.
  *   - `ws` is a caller-owned device workspace of at least lisa_workspace_size(desc) bytes, 256-byte
  *     aligned, zeroed once with lisa_workspace_init before first use.  Its first 256 bytes hold the
  *     error word; the rest is scratch.  Calls that share one workspace must not overlap in time.

@@ -212,8 +212,20 @@ def linear_branch(S, z, k_new, v_new, gate_logit) -> LinearBranch:
     return lb
 
 
-def stage_events(start=None, after_index=None, after_attn=None, end=None) -> StageEvents:
-    h = lambda e: None if e is None else e.cuda_event
+def stage_events(start=None, after_index=None, after_attn=None, end=None, stream=None) -> StageEvents:
+    """Stage events for lisa_fused_decode from torch.cuda.Event objects.
+
+    torch creates the underlying CUDA event lazily, on its first record; each event is
+    recorded once here so that it exists (the library re-records it at its stage).
+    """
+
+    def h(e):
+        if e is None:
+            return None
+        if e.cuda_event == 0:
+            e.record(stream if stream is not None else torch.cuda.current_stream())
+        return e.cuda_event
+
     ev = StageEvents(h(start), h(after_index), h(after_attn), h(end))
     ev._refs = (start, after_index, after_attn, end)
     return ev

@@ -22,8 +22,9 @@ inline int ilog2(int x) {
 }
 
 struct Layout {
-  int G = 0, splits = 0, split_len = 0, chunk_max = 0;
-  size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0, total = 0;
+  int G = 0, splits = 0, split_len = 0, chunk_max = 0, cap = 0;
+  size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0;
+  size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_cand = 0, total = 0;
 };
 
 // Host checks shared by every entry point.  Returns LISA_OK for a valid desc (also when B == 0).
@@ -74,6 +75,16 @@ Layout layout_of(const lisa_decode_desc& d) {
   off += align256(B * Hkv * (size_t)L.splits * L.G * (size_t)d.head_dim * 4);
   L.off_ml = off;
   off += align256(B * Hkv * (size_t)L.splits * L.G * 2 * 4);
+  // Candidate buffer of the fused top-M: room for ~4M keys above the sampled threshold.
+  L.cap = d.max_seq_len < 4 * d.budget_m + 4096 ? d.max_seq_len : 4 * d.budget_m + 4096;
+  L.off_uq = off;
+  off += align256(B * Hkv * 32 * 4);
+  L.off_tau = off;
+  off += align256(B * Hkv * 4);
+  L.off_ccount = off;
+  off += align256(B * Hkv * 4);
+  L.off_cand = off;
+  off += align256(B * Hkv * (size_t)L.cap * 8);
   L.total = off;
   return L;
 }
@@ -99,8 +110,10 @@ lisa_status bind_device(const void* ptr) {
 
 inline lisa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? LISA_OK : LISA_ERR_CUDA; }
 
-// Pointers read with 16-byte vector loads or cp.async must be 16-byte aligned.
+// Pointers read with vector loads or cp.async must be aligned to the access width: 32 bytes for the
+// projected-key pool (256-bit loads), 16 bytes for the K/V pools (16-byte cp.async).
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
@@ -117,9 +130,15 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   p.max_seq_len = d.max_seq_len;
   p.num_pages = d.num_pages;
   p.chunk_max = L.chunk_max;
+  p.cap = L.cap;
   p.seq_lens = d.seq_lens;
   p.page_table = d.page_table;
   p.err = static_cast<uint32_t*>(ws);
+  char* w = static_cast<char*>(ws);
+  p.uq = reinterpret_cast<float*>(w + L.off_uq);
+  p.tau = reinterpret_cast<uint32_t*>(w + L.off_tau);
+  p.ccount = reinterpret_cast<uint32_t*>(w + L.off_ccount);
+  p.cand = reinterpret_cast<uint32_t*>(w + L.off_cand);
   return p;
 }
 
@@ -219,7 +238,7 @@ lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const 
   if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || scores == nullptr)
     return LISA_ERR_INVALID_ARG;
   if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
-  if (!aligned16(kproj_pool) || !aligned4(q) || !aligned4(scores)) return LISA_ERR_INVALID_ARG;
+  if (!aligned32(kproj_pool) || !aligned4(q) || !aligned4(scores)) return LISA_ERR_INVALID_ARG;
   const Layout L = layout_of(*desc);
   LISA_TRY(check_ws(ws, ws_bytes, L));
   LISA_TRY(bind_device(ws));
@@ -258,7 +277,7 @@ lisa_status lisa_index_topm(const lisa_decode_desc* desc, const void* q, const f
       count == nullptr)
     return LISA_ERR_INVALID_ARG;
   if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
-  if (!aligned16(kproj_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  if (!aligned32(kproj_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
   const Layout L = layout_of(*desc);
   LISA_TRY(check_ws(ws, ws_bytes, L));
   LISA_TRY(bind_device(ws));
@@ -270,7 +289,7 @@ lisa_status lisa_index_topm(const lisa_decode_desc* desc, const void* q, const f
   p.kproj_scale = kproj_scale;
   p.idx = idx;
   p.count = count;
-  return cuda_status(launch_index_select(p, false, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_index_topm(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q, const void* k_pool,
@@ -306,7 +325,7 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
   if (!reuse) {
     LISA_TRY(check_idx_dim(desc));
     if (P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr) return LISA_ERR_INVALID_ARG;
-    if (!aligned16(kproj_pool)) return LISA_ERR_INVALID_ARG;
+    if (!aligned32(kproj_pool)) return LISA_ERR_INVALID_ARG;
     if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
   }
   if (lin != nullptr && (lin->S == nullptr || lin->z == nullptr || lin->k_new == nullptr || lin->v_new == nullptr ||
@@ -331,7 +350,7 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
     p.kproj_scale = kproj_scale;
     p.idx = di;
     p.count = dc;
-    LISA_TRY(cuda_status(launch_index_select(p, false, st)));
+    LISA_TRY(cuda_status(launch_index_topm(p, st)));
     idx = di;
     count = dc;
   }

@@ -6,17 +6,16 @@
 // (a tie at the M-th score goes to the lower position) and reported in ascending order.
 //
 // Design on B200:
-//  * Scoring streams the projected-key cache with 16-byte non-allocating vector loads, several per
-//    thread in flight; a page block of one head (page_size * r bytes) is contiguous.  FP8 is decoded
-//    with the hardware e4m3x2 -> f16x2 conversion and accumulated in fp32 on the CUDA cores (a single
-//    query makes this a matrix-vector product: no tensor-core work to be had).
-//  * Selection is fused with scoring.  A cluster of 8 CTAs owns one (b, KV head); each CTA scores a
-//    contiguous, page-aligned eighth of the context into shared memory as order-preserving uint32
-//    keys and builds a histogram of the top 11 key bits while the loads are in flight.  The eight
-//    histograms are summed through distributed shared memory, the digit that holds the M-th key is
-//    found, and two more passes (11 + 10 bits) pin the exact M-th key.  Each CTA then writes its
-//    selected positions in ascending order at an offset derived from the other CTAs' counts.  No
-//    fp32 score array ever goes to HBM on this path.
+//  * Scoring streams the projected-key cache; each lane owns whole rows (one 256-bit load per
+//    32-byte FP8 row, so a warp reads 1 KB of one page block at a time) and keeps up to eight rows
+//    in flight.  FP8 is decoded with the hardware e4m3x2 -> f16x2 conversion and accumulated with
+//    packed fp32x2 FMAs on the CUDA cores (a single query makes this a matrix-vector product: no
+//    tensor-core work to be had).
+//  * The fused top-M never writes the fp32 scores to HBM: a sampled threshold lets the streaming
+//    kernel keep only ~2M candidates per (b, KV head) (see the sample / stream / finish kernels);
+//    the finish kernel does the exact selection on those, with an exact re-scoring fallback.
+//  * Selection from caller-given scores uses a cluster of 8 CTAs per (b, KV head) with the
+//    histograms reduced over distributed shared memory.
 
 #include <cooperative_groups.h>
 
@@ -29,14 +28,67 @@ namespace lisa {
 
 namespace {
 
+
+constexpr int kCandCap = 2048;  // keys inside the threshold digit kept in a list, per CTA
+constexpr int kTieCap = 64;     // ties at the M-th key resolved from a list, per CTA
+
 template <int R, bool FP8>
 struct RowGeom {
-  static constexpr int kElemBytes = FP8 ? 1 : 4;
-  static constexpr int kRowBytes = R * kElemBytes;        // 16, 32, 64 or 128
-  static constexpr int kLanesPerRow = kRowBytes / 16;     // 1, 2, 4, 8
-  static constexpr int kRowsPerLoad = 32 / kLanesPerRow;  // rows one warp-wide 16-byte load covers
-  static constexpr int kElemsPerLane = 16 / kElemBytes;   // elements in one 16-byte load
+  static constexpr int kRowBytes = R * (FP8 ? 1 : 4);     // 16, 32, 64 or 128
+  static constexpr int kVec = kRowBytes >= 32 ? 32 : 16;  // bytes per vector load
+  static constexpr int kLoads = kRowBytes / kVec;         // vector loads per row
+  static constexpr int kWords = kRowBytes / 4;
+  static constexpr int kUnroll = 64 / kWords > 8 ? 8 : 64 / kWords;  // rows in flight per lane
 };
+
+template <int BYTES>
+__device__ __forceinline__ void load_vec(const uint8_t* p, uint32_t* w);
+template <>
+__device__ __forceinline__ void load_vec<32>(const uint8_t* p, uint32_t* w) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+               : "l"(p));
+}
+template <>
+__device__ __forceinline__ void load_vec<16>(const uint8_t* p, uint32_t* w) {
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+               : "l"(p));
+}
+
+// c = a * b + c on two fp32 lanes at once (sm_100 packed FMA).
+__device__ __forceinline__ void ffma2(float2& c, float2 a, float2 b) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\tmov.b64 {%0, %1}, rc;\n\t}\n"
+      : "+f"(c.x), "+f"(c.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+}
+
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_bytes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_bytes, __NV_E4M3);
+  return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+
+// <u, row> for one row held in registers (element e of the row pairs with u[e]).
+template <int R, bool FP8>
+__device__ __forceinline__ float row_dot(const uint32_t* w, const float2* u2) {
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+  if constexpr (FP8) {
+#pragma unroll
+    for (int i = 0; i < R / 4; ++i) {
+      ffma2(a0, e4m3x2_to_float2(w[i] & 0xffffu), u2[2 * i]);
+      ffma2(a1, e4m3x2_to_float2(w[i] >> 16), u2[2 * i + 1]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < R / 4; ++i) {
+      ffma2(a0, make_float2(__uint_as_float(w[4 * i]), __uint_as_float(w[4 * i + 1])), u2[2 * i]);
+      ffma2(a1, make_float2(__uint_as_float(w[4 * i + 2]), __uint_as_float(w[4 * i + 3])), u2[2 * i + 1]);
+    }
+  }
+  return (a0.x + a1.x) + (a0.y + a1.y);
+}
 
 __device__ __forceinline__ int load_seq_len(const IndexParams& p, int b) {
   int n = p.seq_lens[b];
@@ -67,69 +119,6 @@ __device__ void compute_projected_query(const IndexParams& p, int b, int h, floa
   __syncthreads();
 }
 
-template <bool FP8>
-__device__ __forceinline__ float dot16(const uint4& v, const float* uf) {
-  if constexpr (FP8) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3);
-      __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
-      const float2 flo = __half22float2(*reinterpret_cast<__half2*>(&lo));
-      const float2 fhi = __half22float2(*reinterpret_cast<__half2*>(&hi));
-      a0 = fmaf(flo.x, uf[4 * i + 0], a0);
-      a1 = fmaf(flo.y, uf[4 * i + 1], a1);
-      a0 = fmaf(fhi.x, uf[4 * i + 2], a0);
-      a1 = fmaf(fhi.y, uf[4 * i + 3], a1);
-    }
-    return a0 + a1;
-  } else {
-    float a = __uint_as_float(v.x) * uf[0];
-    a = fmaf(__uint_as_float(v.y), uf[1], a);
-    a = fmaf(__uint_as_float(v.z), uf[2], a);
-    a = fmaf(__uint_as_float(v.w), uf[3], a);
-    return a;
-  }
-}
-
-// Score rows [t_begin, t_begin + nrows) of (b, h); t_begin is page aligned and pages[i] holds the
-// (checked) page id of the i-th page of the range.  sink(local_row, score) runs on one lane per row.
-template <int R, bool FP8, int U, class Sink>
-__device__ __forceinline__ void stream_scores(const IndexParams& p, int h, int t_begin, int nrows,
-                                              const int32_t* pages, const float* u, float scale, Sink sink) {
-  using Geo = RowGeom<R, FP8>;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int part = lane % Geo::kLanesPerRow, rsub = lane / Geo::kLanesPerRow;
-  float uf[Geo::kElemsPerLane];
-#pragma unroll
-  for (int e = 0; e < Geo::kElemsPerLane; ++e) uf[e] = u[part * Geo::kElemsPerLane + e];
-  const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
-  const int per_warp_iter = Geo::kRowsPerLoad * U;
-  for (int r0 = warp * per_warp_iter; r0 < nrows; r0 += nwarps * per_warp_iter) {
-    uint4 v[U];
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const int lr = r0 + k * Geo::kRowsPerLoad + rsub;
-      if (lr < nrows) {
-        const int t = t_begin + lr;
-        const size_t row = (((size_t)pages[lr >> p.log2ps] * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1));
-        v[k] = ldg_stream_16(base + row * Geo::kRowBytes + part * 16);
-      } else {
-        v[k] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < U; ++k) {
-      float dot = dot16<FP8>(v[k], uf);
-#pragma unroll
-      for (int o = Geo::kLanesPerRow / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      const int lr = r0 + k * Geo::kRowsPerLoad + rsub;
-      if (part == 0 && lr < nrows) sink(lr, scale * dot);
-    }
-  }
-}
-
 // Checked page ids of pages [first_page, first_page + count) of sequence b.
 __device__ __forceinline__ void load_pages(const IndexParams& p, int b, int first_page, int count, int32_t* pages) {
   for (int i = threadIdx.x; i < count; i += blockDim.x) {
@@ -142,198 +131,136 @@ __device__ __forceinline__ void load_pages(const IndexParams& p, int b, int firs
   }
 }
 
-// Block-wide: among the nb bins of gh (counts of candidate keys per digit, high digit = high key),
-// find the digit d holding the need-th largest candidate.  Writes d and the rank of that key within
-// the digit (1-based) to out[0], out[1].  Ends with a barrier.
-__device__ void find_digit(const uint32_t* gh, int nb, uint32_t need, uint32_t* warp_tot, uint32_t* out) {
+// Score rows [t_begin, t_begin + nrows) of (b, h); t_begin is page aligned and pages[i] holds the
+// checked page id of the i-th page of the range.  Lane l of a warp owns row l of each 32-row group.
+// sink(local_row, score) runs once per row.
+template <int R, bool FP8, class Sink>
+__device__ __forceinline__ void stream_scores(const IndexParams& p, int h, int t_begin, int nrows,
+                                              const int32_t* pages, const float* u, float scale, Sink sink) {
+  using Geo = RowGeom<R, FP8>;
+  constexpr int U = Geo::kUnroll;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  float2 u2[R / 2];
+#pragma unroll
+  for (int k = 0; k < R / 2; ++k) u2[k] = make_float2(u[2 * k], u[2 * k + 1]);
+  const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
+  for (int g0 = warp * U * 32; g0 < nrows; g0 += nwarps * U * 32) {
+    uint32_t w[U][Geo::kWords];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int lr = g0 + k * 32 + lane;
+      if (lr < nrows) {
+        const int t = t_begin + lr;
+        const size_t row = (((size_t)pages[lr >> p.log2ps] * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1));
+        const uint8_t* src = base + row * Geo::kRowBytes;
+#pragma unroll
+        for (int l = 0; l < Geo::kLoads; ++l) load_vec<Geo::kVec>(src + l * Geo::kVec, &w[k][l * (Geo::kVec / 4)]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < Geo::kWords; ++i) w[k][i] = 0u;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int lr = g0 + k * 32 + lane;
+      const float dot = row_dot<R, FP8>(w[k], u2);
+      if (lr < nrows) sink(lr, scale * dot);
+    }
+  }
+}
+
+struct SelectSmem {
+  uint32_t hist0[kBins];      // top 11 key bits
+  uint32_t hist1[kBins];      // next 11 bits, keys inside the pass-0 digit
+  uint32_t hist2[kBins / 2];  // last 10 bits
+  uint32_t cand_key[kCandCap];
+  uint32_t cand_pos[kCandCap];
+  uint32_t tie_pos[kTieCap];
+  uint32_t scan[32];
+  uint32_t digit[2];
+  uint32_t cnt[2];  // (#keys > K, #keys == K) of this CTA, read by the other CTAs of the cluster
+  uint32_t ncand, nabove, ngt, ntie;
+};
+
+// Sum of the cluster's histograms over this thread's PER consecutive bins, into registers.
+template <int PER>
+__device__ __forceinline__ void cluster_bins(cg::cluster_group& cluster, uint32_t* hist, uint32_t (&v)[PER]) {
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = 0u;
+#pragma unroll
+  for (int r = 0; r < kClusterSize; ++r) {
+    const uint4* rh = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, r) + threadIdx.x * PER);
+#pragma unroll
+    for (int q = 0; q < PER / 4; ++q) {
+      const uint4 a = rh[q];
+      v[4 * q + 0] += a.x;
+      v[4 * q + 1] += a.y;
+      v[4 * q + 2] += a.z;
+      v[4 * q + 3] += a.w;
+    }
+  }
+}
+
+// Block-wide: the bins (PER per thread, thread t owns bins [t*PER, (t+1)*PER), higher bin = larger
+// key) hold candidate counts; find the bin holding the need-th largest candidate.  Writes the bin
+// and the rank of that key inside it (1-based) to digit[0..1].  Ends with a barrier.
+template <int PER>
+__device__ void find_digit(const uint32_t (&v)[PER], uint32_t need, uint32_t* scan, uint32_t* digit) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
-  const int per = nb / blockDim.x;
-  uint32_t v = 0;
-  for (int i = 0; i < per; ++i) v += gh[t * per + i];
-  uint32_t x = v;  // inclusive suffix sum within the warp (lanes >= this lane)
+  uint32_t tot = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) tot += v[i];
+  uint32_t x = tot;  // suffix sum over lanes >= this lane
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_down_sync(0xffffffffu, x, o);
     if (lane + o < 32) x += y;
   }
-  if (lane == 0) warp_tot[warp] = x;
+  if (lane == 0) scan[warp] = x;
   __syncthreads();
   uint32_t above = 0;
-  for (int w = warp + 1; w < nwarps; ++w) above += warp_tot[w];
-  const uint32_t incl = x + above, excl = incl - v;
+  for (int w = warp + 1; w < nwarps; ++w) above += scan[w];
+  const uint32_t incl = x + above, excl = incl - tot;
   if (excl < need && need <= incl) {
     uint32_t acc = excl;
-    for (int i = per - 1; i >= 0; --i) {
-      const uint32_t c = gh[t * per + i];
-      if (acc + c >= need) {
-        out[0] = (uint32_t)(t * per + i);
-        out[1] = need - acc;
-        break;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      if (acc < need && acc + v[i] >= need) {
+        digit[0] = (uint32_t)(t * PER + i);
+        digit[1] = need - acc;
       }
-      acc += c;
+      acc += v[i];
     }
   }
   __syncthreads();
 }
 
-struct SelectSmem {
-  uint32_t hist[3][kBins];
-  uint32_t ghist[kBins];
-  float qbar[128];
-  float u[32];
-  uint32_t warp_tot[32];
-  uint32_t digit[2];
-  uint32_t cnt[2];     // this CTA's (#keys > K, #keys == K), read by the other CTAs of the cluster
-  uint32_t wgt[32], weq[32];
-};
-
-}  // namespace
-
-size_t select_smem_bytes(int chunk_max, int ps) {
-  const int pages = (chunk_max + ps - 1) / ps;
-  return sizeof(SelectSmem) + (size_t)chunk_max * 4 + (size_t)pages * 4;
-}
-
-// One cluster of kClusterSize CTAs per (b, KV head).  FROM_SCORES: keys come from p.scores
-// (lisa_topm_select); otherwise the CTA computes them (lisa_index_topm / lisa_fused_decode).
-template <int R, bool FP8, bool FROM_SCORES>
-__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kIndexThreads, 2)
-    lisa_index_select_kernel(IndexParams p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
-  int32_t* pages = reinterpret_cast<int32_t*>(keys + p.chunk_max);
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-  const int n = load_seq_len(p, b);
-  int32_t* idx_out = p.idx + ((size_t)b * p.Hkv + h) * p.M;
-
-  if (n <= p.M) {  // every position is kept; the whole cluster takes this branch together
-    for (int i = rank * blockDim.x + tid; i < p.M; i += kClusterSize * blockDim.x) idx_out[i] = i < n ? i : -1;
-    if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = n;
-    return;
-  }
-
-  // This CTA's page-aligned slice of the context.
-  const int chunk = ((((n + kClusterSize - 1) / kClusterSize) + p.ps - 1) >> p.log2ps) << p.log2ps;
-  const int t_begin = rank * chunk;
-  const int nrows = max(0, min(n, t_begin + chunk) - t_begin);
-
-  for (int i = tid; i < 3 * kBins; i += blockDim.x) (&sm.hist[0][0])[i] = 0u;
-  if constexpr (!FROM_SCORES) {
-    load_pages(p, b, t_begin >> p.log2ps, (nrows + p.ps - 1) >> p.log2ps, pages);
-    compute_projected_query(p, b, h, sm.qbar, sm.u);  // ends with a barrier
-    const float scale = p.kproj_scale[h];
-    stream_scores<R, FP8, 8>(p, h, t_begin, nrows, pages, sm.u, scale, [&](int lr, float s) {
-      const uint32_t k = score_key(s);
-      keys[lr] = k;
-      atomicAdd(&sm.hist[0][k >> 21], 1u);
-    });
-  } else {
-    __syncthreads();
-    const float* src = p.scores + ((size_t)b * p.Hkv + h) * p.max_seq_len + t_begin;
-    for (int lr = tid; lr < nrows; lr += blockDim.x) {
-      const uint32_t k = score_key(src[lr]);
-      keys[lr] = k;
-      atomicAdd(&sm.hist[0][k >> 21], 1u);
-    }
-  }
-
-  // Radix select of the M-th largest key over the cluster: digits of 11, 11 and 10 bits.
-  const int shift[3] = {21, 10, 0};
-  const int width[3] = {11, 11, 10};
-  uint32_t prefix = 0, need = (uint32_t)p.M;
-  for (int pass = 0; pass < 3; ++pass) {
-    uint32_t* hp = sm.hist[pass];
-    if (pass > 0) {
-      const int hs = shift[pass - 1];
-      const uint32_t mask = (1u << width[pass]) - 1u;
-      for (int lr = tid; lr < nrows; lr += blockDim.x) {
-        const uint32_t k = keys[lr];
-        if ((k >> hs) == prefix) atomicAdd(&hp[(k >> shift[pass]) & mask], 1u);
-      }
-    }
-    cluster.sync();  // every CTA's histogram of this pass is complete
-    const int nb = 1 << width[pass];
-    for (int i = tid; i < nb; i += blockDim.x) {
-      uint32_t s = 0;
+// Block-wide exclusive prefix sum of one value per thread; returns the sum over lower threads.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nwarps = blockDim.x >> 5;
+  uint32_t x = v;
 #pragma unroll
-      for (int r = 0; r < kClusterSize; ++r) s += cluster.map_shared_rank(hp, r)[i];
-      sm.ghist[i] = s;
-    }
-    __syncthreads();
-    find_digit(sm.ghist, nb, need, sm.warp_tot, sm.digit);
-    prefix = (prefix << width[pass]) | sm.digit[0];
-    need = sm.digit[1];
-  }
-  const uint32_t K = prefix;      // the M-th largest key of (b, h)
-  const uint32_t tie_take = need;  // keys equal to K to keep, lowest positions first
-
-  // Count per warp over contiguous row ranges, then place this CTA's rows after the lower ranks'.
-  const int wlen = (((nrows + nwarps - 1) / nwarps) + 31) & ~31;
-  const int w0 = warp * wlen, w1 = min(nrows, w0 + wlen);
-  uint32_t gt = 0, eq = 0;
-  for (int lr = w0 + lane; lr < w1; lr += 32) {
-    const uint32_t k = keys[lr];
-    gt += (k > K);
-    eq += (k == K);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    gt += __shfl_xor_sync(0xffffffffu, gt, o);
-    eq += __shfl_xor_sync(0xffffffffu, eq, o);
-  }
-  if (lane == 0) {
-    sm.wgt[warp] = gt;
-    sm.weq[warp] = eq;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
   __syncthreads();
-  if (tid == 0) {
-    uint32_t a = 0, e = 0;
-    for (int w = 0; w < nwarps; ++w) {
-      a += sm.wgt[w];
-      e += sm.weq[w];
-    }
-    sm.cnt[0] = a;
-    sm.cnt[1] = e;
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  uint32_t below = 0, all = 0;
+  for (int w = 0; w < nwarps; ++w) {
+    const uint32_t s = scratch[w];
+    if (w < warp) below += s;
+    all += s;
   }
-  cluster.sync();
-  uint32_t ties_before = 0, out_before = 0;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t* rc = cluster.map_shared_rank(sm.cnt, r);
-    const uint32_t take = min(rc[1], tie_take > ties_before ? tie_take - ties_before : 0u);
-    out_before += rc[0] + take;
-    ties_before += rc[1];
-  }
-  for (int w = 0; w < warp; ++w) {
-    const uint32_t take = min(sm.weq[w], tie_take > ties_before ? tie_take - ties_before : 0u);
-    out_before += sm.wgt[w] + take;
-    ties_before += sm.weq[w];
-  }
-  const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int base = w0; base < w1; base += 32) {
-    const int lr = base + lane;
-    const bool valid = lr < w1;
-    const uint32_t k = valid ? keys[lr] : 0u;
-    const bool is_gt = valid && k > K;
-    const bool is_eq = valid && k == K;
-    const uint32_t beq = __ballot_sync(0xffffffffu, is_eq);
-    const uint32_t tie_rank = ties_before + __popc(beq & lt_mask);
-    const bool take = is_gt || (is_eq && tie_rank < tie_take);
-    const uint32_t bsel = __ballot_sync(0xffffffffu, take);
-    const uint32_t slot = out_before + __popc(bsel & lt_mask);
-    if (take && slot < (uint32_t)p.M) idx_out[slot] = t_begin + lr;
-    ties_before += __popc(beq);
-    out_before += __popc(bsel);
-  }
-  if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = p.M;
-  cluster.sync();  // no CTA leaves while another may still read its counters
+  if (total) *total = all;
+  return below + x - v;
 }
 
+
+// ---------------------------------------------------------------------------------------------
 // Scores only: one CTA per (kScoreChunk positions, KV head, sequence); writes fp32 scores.
+// ---------------------------------------------------------------------------------------------
 template <int R, bool FP8>
 __global__ void __launch_bounds__(kIndexThreads) lisa_score_kernel(IndexParams p) {
   __shared__ float qbar[128];
@@ -347,8 +274,533 @@ __global__ void __launch_bounds__(kIndexThreads) lisa_score_kernel(IndexParams p
   load_pages(p, b, t_begin >> p.log2ps, (nrows + p.ps - 1) >> p.log2ps, pages);
   compute_projected_query(p, b, h, qbar, u);
   float* dst = p.scores + ((size_t)b * p.Hkv + h) * p.max_seq_len + t_begin;
-  stream_scores<R, FP8, 8>(p, h, t_begin, nrows, pages, u, p.kproj_scale[h],
-                           [&](int lr, float s) { dst[lr] = s; });
+  stream_scores<R, FP8>(p, h, t_begin, nrows, pages, u, p.kproj_scale[h], [&](int lr, float s) { dst[lr] = s; });
+}
+
+// ---------------------------------------------------------------------------------------------
+// Top-M with the scores kept on chip, in three steps per (b, KV head):
+//   sample -- project the averaged query (u, kept for the other two steps) and score a strided
+//             sample of up to kSampleMax positions; the threshold key tau is the lower edge of the
+//             top-11-bit bin that holds the ceil(2 M S / n) + 16-th largest sample, so that about
+//             2M positions are expected at or above it;
+//   stream -- score every position and keep (key, position) of those at or above tau: staged in
+//             shared memory, appended to the candidate buffer with one global atomic per CTA;
+//   finish -- exact radix select of the M-th key among the candidates, ties to the lowest
+//             positions, emitted in ascending order from a position bitmap.
+// Exactness: if at least M candidates arrive, the M-th largest key is >= tau, so every position
+// of the top M (ties included) is a candidate.  If fewer arrive, or the buffer overflows, finish
+// recomputes that (b, KV head) exactly by re-scoring all its positions (same arithmetic).
+// ---------------------------------------------------------------------------------------------
+
+// Load the projected-key row of position t of (b, h) (page id checked).
+template <int R, bool FP8>
+__device__ __forceinline__ void load_row(const IndexParams& p, int b, int h, int t, uint32_t* w) {
+  using Geo = RowGeom<R, FP8>;
+  int pg = p.page_table[(size_t)b * p.max_pages + (t >> p.log2ps)];
+  if (pg < 0 || pg >= p.num_pages) {
+    flag_error(p.err, LISA_DEVERR_PAGE_ID);
+    pg = 0;
+  }
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kproj) +
+                       ((((size_t)pg * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1))) * Geo::kRowBytes;
+#pragma unroll
+  for (int l = 0; l < Geo::kLoads; ++l) load_vec<Geo::kVec>(src + l * Geo::kVec, &w[l * (Geo::kVec / 4)]);
+}
+
+template <int R>
+__device__ __forceinline__ void load_u2(const float* u, float2* u2) {
+#pragma unroll
+  for (int k = 0; k < R / 2; ++k) u2[k] = make_float2(u[2 * k], u[2 * k + 1]);
+}
+
+constexpr int kSampleThreads = 512;
+
+template <int R, bool FP8>
+__global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(IndexParams p) {
+  __shared__ float qbar[128];
+  __shared__ float u[32];
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t scan[32];
+  __shared__ uint32_t digit[2];
+  using Geo = RowGeom<R, FP8>;
+  constexpr int kSampleUnroll = Geo::kWords >= 32 ? 1 : 32 / Geo::kWords;  // rows in flight per thread
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const int n = load_seq_len(p, b);
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  compute_projected_query(p, b, h, qbar, u);  // ends with a barrier
+  if (tid < p.r) p.uq[bh * 32 + tid] = u[tid];
+  if (n <= p.M) {
+    if (tid == 0) {
+      p.tau[bh] = 0u;
+      p.ccount[bh] = 0u;
+    }
+    return;
+  }
+  float2 u2[R / 2];
+  load_u2<R>(u, u2);
+  const float scale = p.kproj_scale[h];
+  const int S = min(n, kSampleMax);
+  for (int j0 = tid; j0 < S; j0 += kSampleThreads * kSampleUnroll) {
+    uint32_t w[kSampleUnroll][Geo::kWords];
+#pragma unroll
+    for (int k = 0; k < kSampleUnroll; ++k) {
+      const int j = j0 + k * kSampleThreads;
+      if (j < S) load_row<R, FP8>(p, b, h, (int)(((long long)j * n) / S), w[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kSampleUnroll; ++k) {
+      if (j0 + k * kSampleThreads < S) atomicAdd(&hist[score_key(scale * row_dot<R, FP8>(w[k], u2)) >> 21], 1u);
+    }
+  }
+  __syncthreads();
+  const uint32_t rank = (uint32_t)min((long long)S, (2LL * p.M * S + n - 1) / n + 16);
+  constexpr int PER = kBins / kSampleThreads;
+  uint32_t v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, rank, scan, digit);
+  if (tid == 0) {
+    p.tau[bh] = digit[0] << 21;
+    p.ccount[bh] = 0u;
+  }
+}
+
+template <int R, bool FP8>
+__global__ void __launch_bounds__(kIndexThreads, 2) lisa_index_stream_kernel(IndexParams p) {
+  __shared__ int32_t pages[kScoreChunk / 16];
+  __shared__ uint32_t ckey[kStageCap];
+  __shared__ uint32_t cpos[kStageCap];
+  __shared__ uint32_t s_ncand, s_base;
+  using Geo = RowGeom<R, FP8>;
+  constexpr int U = Geo::kUnroll;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const int n = load_seq_len(p, b);
+  if (n <= p.M) return;
+  const int t_begin = blockIdx.x * kScoreChunk;
+  if (t_begin >= n) return;
+  const int nrows = min(n - t_begin, kScoreChunk);
+  if (tid == 0) s_ncand = 0u;
+  load_pages(p, b, t_begin >> p.log2ps, (nrows + p.ps - 1) >> p.log2ps, pages);
+  const uint32_t tau = p.tau[bh];
+  const float scale = p.kproj_scale[h];
+  float2 u2[R / 2];
+  load_u2<R>(p.uq + bh * 32, u2);
+  __syncthreads();
+
+  const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
+  for (int g0 = warp * U * 32; g0 < nrows; g0 += nwarps * U * 32) {
+    uint32_t w[U][Geo::kWords];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int lr = g0 + k * 32 + lane;
+      if (lr < nrows) {
+        const int t = t_begin + lr;
+        const size_t row = (((size_t)pages[lr >> p.log2ps] * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1));
+        const uint8_t* src = base + row * Geo::kRowBytes;
+#pragma unroll
+        for (int l = 0; l < Geo::kLoads; ++l) load_vec<Geo::kVec>(src + l * Geo::kVec, &w[k][l * (Geo::kVec / 4)]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < Geo::kWords; ++i) w[k][i] = 0u;
+      }
+    }
+    uint32_t key[U];
+    uint32_t mask = 0u;
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      key[k] = score_key(scale * row_dot<R, FP8>(w[k], u2));
+      if (g0 + k * 32 + lane < nrows && key[k] >= tau) mask |= 1u << k;
+    }
+    if (__ballot_sync(0xffffffffu, mask != 0u)) {
+      const uint32_t mine = __popc(mask);
+      uint32_t incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t slot = 0u;
+      if (lane == 31) slot = atomicAdd(&s_ncand, incl);
+      slot = __shfl_sync(0xffffffffu, slot, 31) + incl - mine;
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        if ((mask >> k) & 1u) {
+          if (slot < (uint32_t)kStageCap) {
+            ckey[slot] = key[k];
+            cpos[slot] = (uint32_t)(t_begin + g0 + k * 32 + lane);
+          }
+          ++slot;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t nc = s_ncand;
+  if (nc == 0u) return;
+  if (tid == 0) s_base = atomicAdd(&p.ccount[bh], nc <= (uint32_t)kStageCap ? nc : (uint32_t)p.cap + 1u);
+  __syncthreads();
+  if (nc > (uint32_t)kStageCap) return;  // the count now exceeds the capacity: finish recomputes
+  uint2* dst = reinterpret_cast<uint2*>(p.cand) + bh * (size_t)p.cap;
+  for (uint32_t i = tid; i < nc; i += blockDim.x) {
+    const uint32_t slot = s_base + i;
+    if (slot < (uint32_t)p.cap) dst[slot] = make_uint2(ckey[i], cpos[i]);
+  }
+}
+
+constexpr int kFinishThreads = 512;
+
+}  // namespace
+
+size_t select_smem_bytes(int chunk_max, int ps) {
+  (void)ps;
+  return sizeof(SelectSmem) + (size_t)chunk_max * 4 + (size_t)((chunk_max + 31) / 32) * 4;
+}
+
+// Top-M from caller-given fp32 scores (lisa_topm_select): one cluster of kClusterSize CTAs per
+// (b, KV head).  Each CTA loads a contiguous, page-aligned eighth of the scores into shared memory
+// as order-preserving uint32 keys with a histogram of the top 11 key bits; the histograms are
+// summed through distributed shared memory, one pass over the keys writes a bitmap of the keys
+// above the threshold digit and a list of the keys inside it, two more histogram passes pin the
+// exact M-th key, and each CTA emits its selected positions in ascending order.
+__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kIndexThreads, 2)
+    lisa_select_from_scores_kernel(IndexParams p) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
+  uint32_t* bitmap = keys + p.chunk_max;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int n = load_seq_len(p, b);
+  int32_t* idx_out = p.idx + ((size_t)b * p.Hkv + h) * p.M;
+
+  if (n <= p.M) {  // every position is kept; the whole cluster takes this branch together
+    for (int i = rank * blockDim.x + tid; i < p.M; i += kClusterSize * blockDim.x) idx_out[i] = i < n ? i : -1;
+    if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = n;
+    return;
+  }
+
+  // This CTA's page-aligned slice of the context.
+  const int chunk = ((((n + kClusterSize - 1) / kClusterSize) + p.ps - 1) >> p.log2ps) << p.log2ps;
+  const int t_begin = rank * chunk;
+  const int nrows = max(0, min(n, t_begin + chunk) - t_begin);
+  const int nwords = (nrows + 31) >> 5;
+
+  for (int i = tid; i < kBins; i += blockDim.x) {
+    sm.hist0[i] = 0u;
+    sm.hist1[i] = 0u;
+    if (i < kBins / 2) sm.hist2[i] = 0u;
+  }
+  if (tid == 0) sm.ncand = sm.nabove = sm.ngt = sm.ntie = 0u;
+  __syncthreads();
+  const float* src = p.scores + ((size_t)b * p.Hkv + h) * p.max_seq_len + t_begin;
+  for (int lr = tid; lr < nrows; lr += blockDim.x) {
+    const uint32_t k = score_key(src[lr]);
+    keys[lr] = k;
+    atomicAdd(&sm.hist0[k >> 21], 1u);
+  }
+
+  // ---- pass 0: digit of the top 11 key bits holding the M-th key of (b, h)
+  cluster.sync();
+  {
+    uint32_t v[kBins / kIndexThreads];
+    cluster_bins(cluster, sm.hist0, v);
+    find_digit(v, (uint32_t)p.M, sm.scan, sm.digit);
+  }
+  const uint32_t d0 = sm.digit[0];
+  uint32_t need = sm.digit[1];
+
+  // One pass over the keys: bitmap words of keys above d0, list of keys inside d0.
+  const int wpw = (nwords + nwarps - 1) / nwarps;
+  {
+    uint32_t above = 0;
+    const int wb = warp * wpw, we = min(nwords, wb + wpw);
+    for (int word = wb; word < we; ++word) {
+      const int lr = word * 32 + lane;
+      const bool valid = lr < nrows;
+      const uint32_t k = valid ? keys[lr] : 0u;
+      const uint32_t dig = k >> 21;
+      const uint32_t bal = __ballot_sync(0xffffffffu, valid && dig > d0);
+      if (lane == 0) bitmap[word] = bal;
+      above += __popc(bal);
+      const bool cand = valid && dig == d0;
+      const uint32_t bc = __ballot_sync(0xffffffffu, cand);
+      if (bc) {
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sm.ncand, (uint32_t)__popc(bc));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (cand) {
+          const uint32_t slot = base + __popc(bc & lt_mask);
+          if (slot < (uint32_t)kCandCap) {
+            sm.cand_key[slot] = k;
+            sm.cand_pos[slot] = (uint32_t)lr;
+          }
+        }
+      }
+    }
+    if (lane == 0 && above) atomicAdd(&sm.nabove, above);
+  }
+  __syncthreads();
+  const uint32_t ncand = sm.ncand;
+  const bool listed = ncand <= (uint32_t)kCandCap;
+
+  // ---- pass 1: next 11 bits among keys inside d0
+  if (listed) {
+    for (uint32_t i = tid; i < ncand; i += blockDim.x) atomicAdd(&sm.hist1[(sm.cand_key[i] >> 10) & 0x7ffu], 1u);
+  } else {
+    for (int lr = tid; lr < nrows; lr += blockDim.x) {
+      const uint32_t k = keys[lr];
+      if ((k >> 21) == d0) atomicAdd(&sm.hist1[(k >> 10) & 0x7ffu], 1u);
+    }
+  }
+  cluster.sync();
+  {
+    uint32_t v[kBins / kIndexThreads];
+    cluster_bins(cluster, sm.hist1, v);
+    find_digit(v, need, sm.scan, sm.digit);
+  }
+  const uint32_t prefix22 = (d0 << 11) | sm.digit[0];
+  need = sm.digit[1];
+
+  // ---- pass 2: last 10 bits
+  if (listed) {
+    for (uint32_t i = tid; i < ncand; i += blockDim.x) {
+      const uint32_t k = sm.cand_key[i];
+      if ((k >> 10) == prefix22) atomicAdd(&sm.hist2[k & 0x3ffu], 1u);
+    }
+  } else {
+    for (int lr = tid; lr < nrows; lr += blockDim.x) {
+      const uint32_t k = keys[lr];
+      if ((k >> 10) == prefix22) atomicAdd(&sm.hist2[k & 0x3ffu], 1u);
+    }
+  }
+  cluster.sync();
+  {
+    uint32_t v[kBins / 2 / kIndexThreads];
+    cluster_bins(cluster, sm.hist2, v);
+    find_digit(v, need, sm.scan, sm.digit);
+  }
+  const uint32_t K = (prefix22 << 10) | sm.digit[0];  // the M-th largest key of (b, h)
+  const uint32_t tie_take = sm.digit[1];               // keys equal to K to keep, lowest positions first
+
+  // Keys inside d0 that are above K join the bitmap; keys equal to K are counted.
+  {
+    uint32_t gt = 0;
+    auto visit = [&](uint32_t k, uint32_t pos) {
+      if (k > K) {
+        atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+        ++gt;
+      } else if (k == K) {
+        const uint32_t slot = atomicAdd(&sm.ntie, 1u);
+        if (slot < (uint32_t)kTieCap) sm.tie_pos[slot] = pos;
+      }
+    };
+    if (listed) {
+      for (uint32_t i = tid; i < ncand; i += blockDim.x) visit(sm.cand_key[i], sm.cand_pos[i]);
+    } else {
+      for (int lr = tid; lr < nrows; lr += blockDim.x) {
+        const uint32_t k = keys[lr];
+        if ((k >> 21) == d0) visit(k, (uint32_t)lr);
+      }
+    }
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    if (lane == 0 && gt) atomicAdd(&sm.ngt, gt);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    sm.cnt[0] = sm.nabove + sm.ngt;
+    sm.cnt[1] = sm.ntie;
+  }
+  cluster.sync();
+  uint32_t ties_before = 0, out_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    const uint32_t* rc = cluster.map_shared_rank(sm.cnt, r);
+    const uint32_t c0 = rc[0], c1 = rc[1];
+    out_before += c0 + min(c1, tie_take > ties_before ? tie_take - ties_before : 0u);
+    ties_before += c1;
+  }
+  const uint32_t ntie = sm.cnt[1];
+  const uint32_t take = min(ntie, tie_take > ties_before ? tie_take - ties_before : 0u);
+
+  // Mark the `take` lowest positions among this CTA's keys equal to K.
+  if (take > 0) {
+    if (ntie <= (uint32_t)kTieCap) {
+      for (uint32_t i = tid; i < ntie; i += blockDim.x) {
+        const uint32_t pos = sm.tie_pos[i];
+        uint32_t below = 0;
+        for (uint32_t j = 0; j < ntie; ++j) below += sm.tie_pos[j] < pos;
+        if (below < take) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
+      }
+    } else {
+      // Many ties: rank them in position order (per-warp contiguous word ranges).
+      const int wb = warp * wpw, we = min(nwords, wb + wpw);
+      uint32_t mine = 0;
+      for (int word = wb; word < we; ++word) {
+        const int lr = word * 32 + lane;
+        mine += __popc(__ballot_sync(0xffffffffu, lr < nrows && keys[lr] == K));
+      }
+      uint32_t* wt = sm.scan;
+      __syncthreads();
+      if (lane == 0) wt[warp] = mine;
+      __syncthreads();
+      uint32_t rank_before = 0;
+      for (int w = 0; w < warp; ++w) rank_before += wt[w];
+      for (int word = wb; word < we; ++word) {
+        const int lr = word * 32 + lane;
+        const bool eq = lr < nrows && keys[lr] == K;
+        const uint32_t be = __ballot_sync(0xffffffffu, eq);
+        if (eq && rank_before + __popc(be & lt_mask) < take) atomicOr(&bitmap[word], 1u << lane);
+        rank_before += __popc(be);
+      }
+    }
+  }
+  __syncthreads();
+
+  // Emit this CTA's selected positions in ascending order from the bitmap.
+  {
+    const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
+    const int wb = tid * wpt, we = min(nwords, wb + wpt);
+    uint32_t mine = 0;
+    for (int word = wb; word < we; ++word) mine += __popc(bitmap[word]);
+    uint32_t slot = out_before + block_exclusive_scan(mine, sm.scan, nullptr);
+    for (int word = wb; word < we; ++word) {
+      uint32_t bits = bitmap[word];
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (slot < (uint32_t)p.M) idx_out[slot] = t_begin + word * 32 + bit;
+        ++slot;
+      }
+    }
+  }
+  if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = p.M;
+  cluster.sync();  // no CTA leaves while another may still read its counters
+}
+
+
+size_t finish_smem_bytes(int max_seq_len) { return (size_t)2 * ((max_seq_len + 31) / 32) * 4; }
+
+template <int R, bool FP8>
+__global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(IndexParams p) {
+  extern __shared__ __align__(16) uint32_t fsm[];
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t scan[32];
+  __shared__ uint32_t digit[2];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const int n = load_seq_len(p, b);
+  int32_t* idx_out = p.idx + bh * p.M;
+  if (n <= p.M) {
+    for (int i = tid; i < p.M; i += blockDim.x) idx_out[i] = i < n ? i : -1;
+    if (tid == 0) p.count[bh] = n;
+    return;
+  }
+  const int nwords = (n + 31) >> 5;
+  uint32_t* sel = fsm;
+  uint32_t* tie = fsm + nwords;
+  for (int i = tid; i < nwords; i += blockDim.x) {
+    sel[i] = 0u;
+    tie[i] = 0u;
+  }
+  const uint32_t cnt = p.ccount[bh];
+  const bool fast = cnt >= (uint32_t)p.M && cnt <= (uint32_t)p.cap;
+  const uint2* cand = reinterpret_cast<const uint2*>(p.cand) + bh * (size_t)p.cap;
+  float2 u2[R / 2];
+  load_u2<R>(p.uq + bh * 32, u2);
+  const float scale = p.kproj_scale[h];
+  // Visit (key, position) of every candidate -- or, on the exact fallback, of every position.
+  auto for_each = [&](auto&& fn) {
+    if (fast) {
+      for (uint32_t i = tid; i < cnt; i += blockDim.x) {
+        const uint2 e = cand[i];
+        fn(e.x, e.y);
+      }
+    } else {
+      for (int t = tid; t < n; t += blockDim.x) {
+        uint32_t w[RowGeom<R, FP8>::kWords];
+        load_row<R, FP8>(p, b, h, t, w);
+        fn(score_key(scale * row_dot<R, FP8>(w, u2)), (uint32_t)t);
+      }
+    }
+  };
+  constexpr int PER = kBins / kFinishThreads;
+  // pass 0: top 11 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) { atomicAdd(&hist[k >> 21], 1u); });
+  __syncthreads();
+  uint32_t v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, (uint32_t)p.M, scan, digit);
+  const uint32_t d0 = digit[0];
+  uint32_t need = digit[1];
+  // pass 1: next 11 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) {
+    if ((k >> 21) == d0) atomicAdd(&hist[(k >> 10) & 0x7ffu], 1u);
+  });
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, need, scan, digit);
+  const uint32_t p22 = (d0 << 11) | digit[0];
+  need = digit[1];
+  // pass 2: last 10 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) {
+    if ((k >> 10) == p22) atomicAdd(&hist[k & 0x3ffu], 1u);
+  });
+  __syncthreads();
+  uint32_t v2[PER / 2];
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i) v2[i] = hist[tid * (PER / 2) + i];
+  find_digit(v2, need, scan, digit);
+  const uint32_t K = (p22 << 10) | digit[0];  // the M-th largest key
+  const uint32_t tie_take = digit[1];         // keys equal to K to keep, lowest positions first
+  for_each([&](uint32_t k, uint32_t pos) {
+    if (k > K)
+      atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    else if (k == K)
+      atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+  });
+  __syncthreads();
+  // Keep the tie_take lowest tied positions; then emit every kept position in ascending order.
+  const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
+  const int wb = tid * wpt, we = min(nwords, wb + wpt);
+  uint32_t mine = 0;
+  for (int i = wb; i < we; ++i) mine += __popc(tie[i]);
+  uint32_t rank = block_exclusive_scan(mine, scan, nullptr);
+  for (int i = wb; i < we && rank < tie_take; ++i) {
+    uint32_t bits = tie[i];
+    while (bits && rank < tie_take) {
+      const uint32_t low = bits & (~bits + 1u);
+      sel[i] |= low;
+      bits ^= low;
+      ++rank;
+    }
+  }
+  mine = 0;
+  for (int i = wb; i < we; ++i) mine += __popc(sel[i]);
+  uint32_t slot = block_exclusive_scan(mine, scan, nullptr);
+  for (int i = wb; i < we; ++i) {
+    uint32_t bits = sel[i];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (slot < (uint32_t)p.M) idx_out[slot] = i * 32 + bit;
+      ++slot;
+    }
+  }
+  if (tid == 0) p.count[bh] = p.M;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -361,30 +813,35 @@ static cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int R, bool FP8>
-static cudaError_t launch_select_t(const IndexParams& p, bool from_scores, cudaStream_t stream) {
+cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream) {
+  (void)from_scores;
   const size_t smem = select_smem_bytes(p.chunk_max, p.ps);
-  dim3 grid(kClusterSize, p.Hkv, p.B);
-  if (from_scores) {
-    auto k = lisa_index_select_kernel<R, FP8, true>;
-    cudaError_t e = set_smem(k, smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kIndexThreads, smem, stream>>>(p);
-  } else {
-    auto k = lisa_index_select_kernel<R, FP8, false>;
-    cudaError_t e = set_smem(k, smem);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kIndexThreads, smem, stream>>>(p);
-  }
+  cudaError_t e = set_smem(lisa_select_from_scores_kernel, smem);
+  if (e != cudaSuccess) return e;
+  lisa_select_from_scores_kernel<<<dim3(kClusterSize, p.Hkv, p.B), kIndexThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream) {
-  if (from_scores) return launch_select_t<32, true>(p, true, stream);  // geometry unused when reading scores
-  if (p.kproj_fp8) {
-    return p.r == 16 ? launch_select_t<16, true>(p, false, stream) : launch_select_t<32, true>(p, false, stream);
-  }
-  return p.r == 16 ? launch_select_t<16, false>(p, false, stream) : launch_select_t<32, false>(p, false, stream);
+template <int R, bool FP8>
+static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream) {
+  lisa_index_sample_kernel<R, FP8><<<dim3(p.Hkv, p.B), kSampleThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const dim3 grid((p.max_seq_len + kScoreChunk - 1) / kScoreChunk, p.Hkv, p.B);
+  lisa_index_stream_kernel<R, FP8><<<grid, kIndexThreads, 0, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = finish_smem_bytes(p.max_seq_len);
+  auto fk = lisa_index_finish_kernel<R, FP8>;
+  e = set_smem(fk, smem);
+  if (e != cudaSuccess) return e;
+  fk<<<dim3(p.Hkv, p.B), kFinishThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream) {
+  if (p.kproj_fp8) return p.r == 16 ? launch_topm_t<16, true>(p, stream) : launch_topm_t<32, true>(p, stream);
+  return p.r == 16 ? launch_topm_t<16, false>(p, stream) : launch_topm_t<32, false>(p, stream);
 }
 
 template <int R, bool FP8>

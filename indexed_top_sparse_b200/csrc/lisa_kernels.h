@@ -8,12 +8,19 @@
 
 namespace lisa {
 
-constexpr int kScoreChunk = 4096;  // positions per CTA of the score-only kernel
+constexpr int kScoreChunk = 4096;   // positions per CTA of the score-only and streaming kernels
+constexpr int kSampleMax = 4096;    // positions the threshold sample scores per (b, KV head)
+constexpr int kStageCap = 1024;     // candidates a streaming CTA can stage in shared memory
 
 struct IndexParams {
   int B, Hq, Hkv, d, r, M, ps, log2ps, max_pages, max_seq_len, num_pages;
   int chunk_max;  // positions per CTA of a select cluster, at most (multiple of ps)
+  int cap;        // candidate-buffer entries per (b, KV head)
   bool kproj_fp8;
+  float* uq;           // [B][Hkv][32]: projected averaged query (written by the sample kernel)
+  uint32_t* tau;       // [B][Hkv]: candidate threshold key
+  uint32_t* ccount;    // [B][Hkv]: candidates appended (may exceed cap: overflow)
+  uint32_t* cand;      // [B][Hkv][cap][2]: (key, position)
   const int32_t* seq_lens;
   const int32_t* page_table;
   const __nv_bfloat16* q;
@@ -61,6 +68,8 @@ size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
+cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream);
+size_t finish_smem_bytes(int max_seq_len);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 

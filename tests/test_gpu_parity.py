@@ -299,9 +299,9 @@ def test_gate_extremes_on_device(cuda_device):
     for g, which in ((60.0, "sparse"), (-60.0, "linear")):
         lin = prob.lin.clone()
         lin.gate.fill_(g)
+        inp = host_inputs(prob, lin=lin)  # before the call: the library updates S and z in place
         ws = R.workspace(prob)
         res = R.fused(prob, ws, lin=lin)
-        inp = host_inputs(prob, lin=lin)
         ref = O.decode_step(inp)
         check_outputs(f64(res["out"]), ref["out"], all_pairs(prob), prob.G)
         if which == "sparse":
@@ -347,3 +347,49 @@ def test_full_size_hybrid_sampled(cuda_device):
         check_outputs(f64(outs[layer]["out"][sel]), refs[layer]["out"], same, prob0.G)
     del lp, outs, state
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------------------------
+# The fused top-M keeps only candidates above a sampled threshold; these inputs defeat the
+# threshold on purpose, so the exact re-scoring path must give the oracle's sets.
+# ---------------------------------------------------------------------------------------------
+
+
+def test_fused_topm_candidate_overflow_falls_back_exactly(cuda_device):
+    # every projected key equal: all scores tie, far more candidates than the buffer holds
+    prob = small(cuda_device, B=2, Hq=8, Hkv=2, M=1024, seq_lens=[20000, 9000], paged=True, seed=95)
+    prob.kproj.fill_(0x38)  # E4M3 1.0
+    ws = R.workspace(prob)
+    idx, count = R.index_topm(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    inp = host_inputs(prob)
+    ref = O.decode_step(inp)
+    for b, h in all_pairs(prob):
+        assert ref["idx"][b][h].tolist() == list(range(1024))
+        assert idx[b, h].tolist() == list(range(1024)) and int(count[b, h]) == 1024
+
+
+def test_fused_topm_too_few_candidates_falls_back_exactly(cuda_device):
+    # High scores only on a few hundred of the positions the threshold sample looks at: the sampled
+    # threshold then sits above the M-th score, fewer than M candidates arrive, and the exact path runs.
+    n, M = 100000, 2048
+    prob = small(cuda_device, B=1, Hq=4, Hkv=2, d=64, r=16, M=M, seq_lens=[n], paged=False, kproj_fp8=False,
+                 plant=("none",), seed=96)
+    S = min(n, 4096)
+    hot = torch.tensor([(j * n) // S for j in range(300)], dtype=torch.long)
+    G = prob.G
+    for h in range(prob.Hkv):
+        qbar = prob.q[0, h * G : (h + 1) * G].double().mean(0)
+        u = prob.P[h].double().cpu() @ qbar.cpu()
+        row = (50.0 * u / (u @ u)).float().to(cuda_device)
+        pages = prob.page_table[0, hot // prob.page_size].long().to(cuda_device)
+        prob.kproj[pages, h, (hot % prob.page_size).to(cuda_device)] = row
+    ws = R.workspace(prob)
+    idx, count = R.index_topm(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    inp = host_inputs(prob)
+    ref = O.decode_step(inp)
+    same = check_index_sets(idx.cpu().numpy(), count.cpu().numpy(), ref, inp["seq_lens"], M, all_pairs(prob))
+    assert len(same) == len(all_pairs(prob))
+    for h in range(prob.Hkv):
+        assert set(hot.tolist()) <= set(idx[0, h].tolist())
