@@ -300,10 +300,10 @@ def run_ours(args, world, rank, local):
             "workload": WORKLOAD if args.batch == 16 else WORKLOAD.replace("B=16", f"B={args.batch}"),
             "sequences_per_gpu": B,
             "l2": "inputs larger than L2 (~671 MB touched per step, 126 MB L2); no flush",
-            "launch": "lisa_fused_decode per step (index+select, split attention, merge)",
+            "launch": "lisa_fused_decode per step: threshold sample, score stream + top-M, split attention + merge",
         },
         "roofline": {
-            "kernel": "lisa_index_select_kernel (FP8 score + cluster top-M)",
+            "kernel": "index stage: lisa_index_sample_kernel + lisa_index_stream_kernel (FP8 score + exact top-M)",
             "bound": "hbm",
             "achieved": achieved,
             "peak": hbm,
@@ -318,7 +318,7 @@ def run_ours(args, world, rank, local):
             "required_bytes_per_step": step_bytes,
             "achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
             "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm,
-            "stage_ms": {"index_select": idx_ms, "attention": attn_ms, "merge": merge_ms},
+            "stage_ms": {"index_select": idx_ms, "attention_and_merge": attn_ms + merge_ms},
         },
         "e2e": {
             "value": B * world / (e2e_ms * 1e-3),

@@ -119,8 +119,9 @@ typedef struct {
 typedef struct {
   lisa_event_t start;       /* before the index stage (score + top-M)         */
   lisa_event_t after_index; /* after the index stage, before attention        */
-  lisa_event_t after_attn;  /* after the split attention, before the merge    */
-  lisa_event_t end;         /* after the merge / linear branch / gate         */
+  lisa_event_t after_attn;  /* after the attention kernel (which also merges the partitions and
+                               applies the linear branch and gate)            */
+  lisa_event_t end;         /* end of the call                                */
 } lisa_stage_events;
 
 /* Workspace bytes any entry point needs for `desc` (0 if desc is invalid). Host only. */

@@ -24,7 +24,7 @@ inline int ilog2(int x) {
 struct Layout {
   int G = 0, splits = 0, split_len = 0, chunk_max = 0, cap = 0;
   size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0;
-  size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_cand = 0, total = 0;
+  size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_done = 0, off_acount = 0, off_cand = 0, total = 0;
 };
 
 // Host checks shared by every entry point.  Returns LISA_OK for a valid desc (also when B == 0).
@@ -77,11 +77,16 @@ Layout layout_of(const lisa_decode_desc& d) {
   off += align256(B * Hkv * (size_t)L.splits * L.G * 2 * 4);
   // Candidate buffer of the fused top-M: room for ~4M keys above the sampled threshold.
   L.cap = d.max_seq_len < 4 * d.budget_m + 4096 ? d.max_seq_len : 4 * d.budget_m + 4096;
+  L.cap = (L.cap + 1) & ~1;  // even: the finish step reads candidates in pairs
   L.off_uq = off;
   off += align256(B * Hkv * 32 * 4);
   L.off_tau = off;
   off += align256(B * Hkv * 4);
   L.off_ccount = off;
+  off += align256(B * Hkv * 4);
+  L.off_done = off;
+  off += align256(B * Hkv * 4);
+  L.off_acount = off;
   off += align256(B * Hkv * 4);
   L.off_cand = off;
   off += align256(B * Hkv * (size_t)L.cap * 8);
@@ -138,12 +143,15 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   p.uq = reinterpret_cast<float*>(w + L.off_uq);
   p.tau = reinterpret_cast<uint32_t*>(w + L.off_tau);
   p.ccount = reinterpret_cast<uint32_t*>(w + L.off_ccount);
+  p.done = reinterpret_cast<uint32_t*>(w + L.off_done);
+  p.acount = reinterpret_cast<uint32_t*>(w + L.off_acount);
   p.cand = reinterpret_cast<uint32_t*>(w + L.off_cand);
   return p;
 }
 
 AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, const void* q, const void* k_pool,
-                       const void* v_pool, const int32_t* idx, const int32_t* count) {
+                       const void* v_pool, const int32_t* idx, const int32_t* count, void* out, float* lse,
+                       const lisa_linear_branch* lin) {
   AttnParams p{};
   p.B = d.batch;
   p.Hq = d.num_q_heads;
@@ -169,33 +177,27 @@ AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, con
   char* w = static_cast<char*>(ws);
   p.o_part = reinterpret_cast<float*>(w + L.off_opart);
   p.ml_part = reinterpret_cast<float*>(w + L.off_ml);
+  p.acount = reinterpret_cast<uint32_t*>(w + L.off_acount);
   p.err = static_cast<uint32_t*>(ws);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  if (lin != nullptr) {
+    p.S = lin->S;
+    p.z = lin->z;
+    p.k_new = static_cast<const __nv_bfloat16*>(lin->k_new);
+    p.v_new = static_cast<const __nv_bfloat16*>(lin->v_new);
+    p.gate = lin->gate_logit;
+  }
   return p;
 }
 
-MergeParams merge_params(const lisa_decode_desc& d, const Layout& L, void* ws, const void* q, void* out, float* lse,
-                         const lisa_linear_branch* lin) {
-  MergeParams m{};
-  m.B = d.batch;
-  m.Hq = d.num_q_heads;
-  m.Hkv = d.num_kv_heads;
-  m.d = d.head_dim;
-  m.splits = L.splits;
-  char* w = static_cast<char*>(ws);
-  m.o_part = reinterpret_cast<const float*>(w + L.off_opart);
-  m.ml_part = reinterpret_cast<const float*>(w + L.off_ml);
-  m.q = static_cast<const __nv_bfloat16*>(q);
-  m.out = static_cast<__nv_bfloat16*>(out);
-  m.lse = lse;
-  if (lin != nullptr) {
-    m.S = lin->S;
-    m.z = lin->z;
-    m.k_new = static_cast<const __nv_bfloat16*>(lin->k_new);
-    m.v_new = static_cast<const __nv_bfloat16*>(lin->v_new);
-    m.gate = lin->gate_logit;
-  }
-  return m;
+// Partition counters start at zero for every attention launch; the fused path's sample kernel
+// clears them, other paths clear them here.
+lisa_status clear_attn_counters(const lisa_decode_desc& d, const Layout& L, void* ws, cudaStream_t st) {
+  return cuda_status(cudaMemsetAsync(static_cast<char*>(ws) + L.off_acount, 0,
+                                     (size_t)d.batch * d.num_kv_heads * 4, st));
 }
+
 
 lisa_status record(lisa_event_t ev, cudaStream_t stream) {
   if (ev == nullptr) return LISA_OK;
@@ -304,8 +306,9 @@ lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q,
   LISA_TRY(check_ws(ws, ws_bytes, L));
   LISA_TRY(bind_device(ws));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  LISA_TRY(cuda_status(launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count), st)));
-  return cuda_status(launch_merge(merge_params(*desc, L, ws, q, out, lse, nullptr), st));
+  LISA_TRY(clear_attn_counters(*desc, L, ws, st));
+  return cuda_status(
+      launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count, out, lse, nullptr), st));
 }
 
 lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,
@@ -353,11 +356,13 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
     LISA_TRY(cuda_status(launch_index_topm(p, st)));
     idx = di;
     count = dc;
+  } else {
+    LISA_TRY(clear_attn_counters(*desc, L, ws, st));
   }
   if (events) LISA_TRY(record(events->after_index, st));
-  LISA_TRY(cuda_status(launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count), st)));
+  LISA_TRY(cuda_status(
+      launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count, out, lse, lin), st)));
   if (events) LISA_TRY(record(events->after_attn, st));
-  LISA_TRY(cuda_status(launch_merge(merge_params(*desc, L, ws, q, out, lse, lin), st)));
   if (events) LISA_TRY(record(events->end, st));
   return LISA_OK;
 }

@@ -46,6 +46,116 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
 
 size_t attn_smem_bytes(int d) { return d == 64 ? AttnGeom<64>::kSmem : AttnGeom<128>::kSmem; }
 
+__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
+
+// Merge the partitions of one (b, KV head) for its G query heads; optional linear branch + gate.
+// Run by the 128 threads of the last partition CTA of (b, h); thread e owns output column e.
+template <int D>
+__device__ void merge_pair(const AttnParams& p, int b, int h) {
+  __shared__ float fk[D];
+  __shared__ float fq[kMaxG][D];
+  __shared__ float zn[D];
+  __shared__ float den[kMaxG];
+  __shared__ float wsplit[kMaxG][64];
+  __shared__ float mstar[kMaxG], lstar[kMaxG];
+  const int G = p.Hq / p.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const float* mlp = p.ml_part + bh * p.splits * G * 2;
+  const float* op = p.o_part + bh * p.splits * G * D;
+
+  // Partition weights, in chunks of 64 partitions.
+  float acc[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  if (tid < G) {
+    float mx = kNegInf;
+    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, __ldcg(&mlp[(s * G + tid) * 2]));
+    float l = 0.f;
+    if (mx != kNegInf)
+      for (int s = 0; s < p.splits; ++s) {
+        const float ms = __ldcg(&mlp[(s * G + tid) * 2]);
+        if (ms != kNegInf) l += __ldcg(&mlp[(s * G + tid) * 2 + 1]) * exp2f(ms - mx);
+      }
+    mstar[tid] = mx;
+    lstar[tid] = l;
+  }
+  for (int s0 = 0; s0 < p.splits; s0 += 64) {
+    __syncthreads();
+    for (int e = tid; e < G * 64; e += blockDim.x) {
+      const int g = e / 64, s = s0 + (e - g * 64);
+      float w = 0.f;
+      if (s < p.splits) {
+        const float ms = __ldcg(&mlp[(s * G + g) * 2]);
+        if (ms != kNegInf && mstar[g] != kNegInf) w = exp2f(ms - mstar[g]);
+      }
+      wsplit[g][e - g * 64] = w;
+    }
+    __syncthreads();
+    if (tid < D) {
+      const int s1 = min(p.splits, s0 + 64);
+      for (int s = s0; s < s1; ++s)
+        for (int g = 0; g < G; ++g) acc[g] += wsplit[g][s - s0] * __ldcg(&op[((size_t)s * G + g) * D + tid]);
+    }
+  }
+  float sparse[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) sparse[g] = (g < G && lstar[g] > 0.f) ? acc[g] / lstar[g] : 0.f;
+  if (p.lse != nullptr && tid < G) {
+    const float l = lstar[tid];
+    p.lse[(size_t)b * p.Hq + (size_t)h * G + tid] =
+        l > 0.f ? (mstar[tid] + log2f(l)) * 0.69314718055994530942f : kNegInf;
+  }
+
+  float outv[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) outv[g] = sparse[g];
+  if (p.S != nullptr) {
+    // Linear branch: S += phi(k) v^T, z += phi(k); lin_g = phi(q_g)^T S / (phi(q_g) . z).
+    if (tid < D) {
+      const float f = phi_elu1(__bfloat162float(p.k_new[bh * D + tid]));
+      fk[tid] = f;
+      zn[tid] = p.z[bh * D + tid] + f;
+      for (int g = 0; g < G; ++g)
+        fq[g][tid] = phi_elu1(__bfloat162float(p.q[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid]));
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += blockDim.x >> 5) {
+      float a = 0.f;
+      for (int c = lane; c < D; c += 32) a = fmaf(fq[g][c], zn[c], a);
+      a = warp_sum(a);
+      if (lane == 0) den[g] = a;
+    }
+    if (tid < D) p.z[bh * D + tid] = zn[tid];
+    __syncthreads();
+    if (tid < D) {
+      float lin[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) lin[g] = 0.f;
+      const float ve = __bfloat162float(p.v_new[bh * D + tid]);
+      float* Sbh = p.S + bh * D * D;
+      for (int c = 0; c < D; ++c) {
+        const float sn = fmaf(fk[c], ve, Sbh[(size_t)c * D + tid]);
+        Sbh[(size_t)c * D + tid] = sn;
+#pragma unroll
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) lin[g] = fmaf(fq[g][c], sn, lin[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) {
+        if (g < G) {
+          const float sg = 1.f / (1.f + expf(-p.gate[(size_t)h * G + g]));
+          outv[g] = sg * sparse[g] + (1.f - sg) * (lin[g] / den[g]);
+        }
+      }
+    }
+  }
+  if (tid < D) {
+    for (int g = 0; g < G; ++g)
+      p.out[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid] = __float2bfloat16_rn(outv[g]);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnParams p) {
   using Geo = AttnGeom<D>;
@@ -255,116 +365,19 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     p.ml_part[(part * G + tid) * 2 + 0] = mx;
     p.ml_part[(part * G + tid) * 2 + 1] = l;
   }
-}
-
-__device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
-
-// Merge the partitions of one (b, KV head) for its G query heads; optional linear branch + gate.
-// One CTA per (KV head, sequence); thread e owns output column e.
-template <int D>
-__global__ void __launch_bounds__(128) lisa_merge_kernel(MergeParams p) {
-  __shared__ float fk[D];
-  __shared__ float fq[kMaxG][D];
-  __shared__ float zn[D];
-  __shared__ float den[kMaxG];
-  __shared__ float wsplit[kMaxG][64];
-  __shared__ float mstar[kMaxG], lstar[kMaxG];
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int G = p.Hq / p.Hkv;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const size_t bh = (size_t)b * p.Hkv + h;
-  const float* mlp = p.ml_part + bh * p.splits * G * 2;
-  const float* op = p.o_part + bh * p.splits * G * D;
-
-  // Partition weights, in chunks of 64 partitions.
-  float acc[kMaxG];
-#pragma unroll
-  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
-  if (tid < G) {
-    float mx = kNegInf;
-    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, mlp[(s * G + tid) * 2]);
-    float l = 0.f;
-    if (mx != kNegInf)
-      for (int s = 0; s < p.splits; ++s) {
-        const float ms = mlp[(s * G + tid) * 2];
-        if (ms != kNegInf) l += mlp[(s * G + tid) * 2 + 1] * exp2f(ms - mx);
-      }
-    mstar[tid] = mx;
-    lstar[tid] = l;
+  // The CTA that completes the last partition of (b, h) merges them (no waiting on other CTAs).
+  __shared__ uint32_t s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const size_t bh = (size_t)b * p.Hkv + h;
+    s_last = atomicAdd(&p.acount[bh], 1u) == (uint32_t)p.splits - 1u;
+    if (s_last) p.acount[bh] = 0u;
   }
-  for (int s0 = 0; s0 < p.splits; s0 += 64) {
-    __syncthreads();
-    for (int e = tid; e < G * 64; e += blockDim.x) {
-      const int g = e / 64, s = s0 + (e - g * 64);
-      float w = 0.f;
-      if (s < p.splits) {
-        const float ms = mlp[(s * G + g) * 2];
-        if (ms != kNegInf && mstar[g] != kNegInf) w = exp2f(ms - mstar[g]);
-      }
-      wsplit[g][e - g * 64] = w;
-    }
-    __syncthreads();
-    if (tid < D) {
-      const int s1 = min(p.splits, s0 + 64);
-      for (int s = s0; s < s1; ++s)
-        for (int g = 0; g < G; ++g) acc[g] += wsplit[g][s - s0] * op[((size_t)s * G + g) * D + tid];
-    }
-  }
-  float sparse[kMaxG];
-#pragma unroll
-  for (int g = 0; g < kMaxG; ++g) sparse[g] = (g < G && lstar[g] > 0.f) ? acc[g] / lstar[g] : 0.f;
-  if (p.lse != nullptr && tid < G) {
-    const float l = lstar[tid];
-    p.lse[(size_t)b * p.Hq + (size_t)h * G + tid] =
-        l > 0.f ? (mstar[tid] + log2f(l)) * 0.69314718055994530942f : kNegInf;
-  }
-
-  float outv[kMaxG];
-#pragma unroll
-  for (int g = 0; g < kMaxG; ++g) outv[g] = sparse[g];
-  if (p.S != nullptr) {
-    // Linear branch: S += phi(k) v^T, z += phi(k); lin_g = phi(q_g)^T S / (phi(q_g) . z).
-    if (tid < D) {
-      const float f = phi_elu1(__bfloat162float(p.k_new[bh * D + tid]));
-      fk[tid] = f;
-      zn[tid] = p.z[bh * D + tid] + f;
-      for (int g = 0; g < G; ++g)
-        fq[g][tid] = phi_elu1(__bfloat162float(p.q[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid]));
-    }
-    __syncthreads();
-    for (int g = warp; g < G; g += blockDim.x >> 5) {
-      float a = 0.f;
-      for (int c = lane; c < D; c += 32) a = fmaf(fq[g][c], zn[c], a);
-      a = warp_sum(a);
-      if (lane == 0) den[g] = a;
-    }
-    if (tid < D) p.z[bh * D + tid] = zn[tid];
-    __syncthreads();
-    if (tid < D) {
-      float lin[kMaxG];
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g) lin[g] = 0.f;
-      const float ve = __bfloat162float(p.v_new[bh * D + tid]);
-      float* Sbh = p.S + bh * D * D;
-      for (int c = 0; c < D; ++c) {
-        const float sn = fmaf(fk[c], ve, Sbh[(size_t)c * D + tid]);
-        Sbh[(size_t)c * D + tid] = sn;
-#pragma unroll
-        for (int g = 0; g < kMaxG; ++g)
-          if (g < G) lin[g] = fmaf(fq[g][c], sn, lin[g]);
-      }
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g) {
-        if (g < G) {
-          const float sg = 1.f / (1.f + expf(-p.gate[(size_t)h * G + g]));
-          outv[g] = sg * sparse[g] + (1.f - sg) * (lin[g] / den[g]);
-        }
-      }
-    }
-  }
-  if (tid < D) {
-    for (int g = 0; g < G; ++g)
-      p.out[((size_t)b * p.Hq + (size_t)h * G + g) * D + tid] = __float2bfloat16_rn(outv[g]);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    merge_pair<D>(p, b, h);
   }
 }
 
@@ -384,13 +397,5 @@ cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream) {
-  dim3 grid(p.Hkv, p.B);
-  if (p.d == 64)
-    lisa_merge_kernel<64><<<grid, 128, 0, stream>>>(p);
-  else
-    lisa_merge_kernel<128><<<grid, 128, 0, stream>>>(p);
-  return cudaGetLastError();
-}
 
 }  // namespace lisa

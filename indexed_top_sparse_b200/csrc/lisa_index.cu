@@ -320,6 +320,7 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   __shared__ float qbar[128];
   __shared__ float u[32];
   __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t skey[kSampleMax];
   __shared__ uint32_t scan[32];
   __shared__ uint32_t digit[2];
   using Geo = RowGeom<R, FP8>;
@@ -330,10 +331,17 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
   compute_projected_query(p, b, h, qbar, u);  // ends with a barrier
   if (tid < p.r) p.uq[bh * 32 + tid] = u[tid];
-  if (n <= p.M) {
+  if (tid == 0) {
+    p.ccount[bh] = 0u;
+    p.done[bh] = 0u;
+    p.acount[bh] = 0u;
+  }
+  if (n <= p.M) {  // every position is kept; the streaming kernel skips this pair
+    int32_t* idx_out = p.idx + bh * p.M;
+    for (int i = tid; i < p.M; i += blockDim.x) idx_out[i] = i < n ? i : -1;
     if (tid == 0) {
       p.tau[bh] = 0u;
-      p.ccount[bh] = 0u;
+      p.count[bh] = n;
     }
     return;
   }
@@ -350,69 +358,282 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
     }
 #pragma unroll
     for (int k = 0; k < kSampleUnroll; ++k) {
-      if (j0 + k * kSampleThreads < S) atomicAdd(&hist[score_key(scale * row_dot<R, FP8>(w[k], u2)) >> 21], 1u);
+      const int j = j0 + k * kSampleThreads;
+      if (j < S) {
+        const uint32_t key = score_key(scale * row_dot<R, FP8>(w[k], u2));
+        skey[j] = key;
+        atomicAdd(&hist[key >> 21], 1u);
+      }
     }
   }
   __syncthreads();
+  // tau: lower edge of the 22-bit key bin that holds the rank-th largest sample key
   const uint32_t rank = (uint32_t)min((long long)S, (2LL * p.M * S + n - 1) / n + 16);
   constexpr int PER = kBins / kSampleThreads;
   uint32_t v[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
   find_digit(v, rank, scan, digit);
-  if (tid == 0) {
-    p.tau[bh] = digit[0] << 21;
-    p.ccount[bh] = 0u;
-  }
+  const uint32_t d0 = digit[0], need = digit[1];
+  __syncthreads();
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for (int j = tid; j < S; j += blockDim.x)
+    if ((skey[j] >> 21) == d0) atomicAdd(&hist[(skey[j] >> 10) & 0x7ffu], 1u);
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, need, scan, digit);
+  if (tid == 0) p.tau[bh] = (d0 << 21) | (digit[0] << 10);
 }
 
+// Exact top-M of (b, h) (n > M) by the whole CTA, from the candidate buffer -- or, when it holds
+// fewer than M candidates or overflowed, by re-scoring every position.  fsm: two bitmaps of
+// ceil(n / 32) words, then room for `stage_cap` candidates staged from global memory.
+template <int R, bool FP8, int THREADS>
+__device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t* fsm, uint32_t* cstage,
+                            uint32_t stage_cap) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t scan[32];
+  __shared__ uint32_t digit[2];
+  const int tid = threadIdx.x;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  int32_t* idx_out = p.idx + bh * p.M;
+  const int nwords = (n + 31) >> 5;
+  uint32_t* sel = fsm;
+  uint32_t* tie = fsm + nwords;
+  for (int i = tid; i < nwords; i += blockDim.x) {
+    sel[i] = 0u;
+    tie[i] = 0u;
+  }
+  const uint32_t cnt = __ldcg(&p.ccount[bh]);
+  const bool fast = cnt >= (uint32_t)p.M && cnt <= (uint32_t)p.cap;
+  const uint2* cand = reinterpret_cast<const uint2*>(p.cand) + bh * (size_t)p.cap;
+  float2 u2[R / 2];
+  load_u2<R>(p.uq + bh * 32, u2);
+  const float scale = p.kproj_scale[h];
+  // Candidates that fit are staged in shared memory once; the passes below then read them there.
+  const bool staged = fast && cnt <= stage_cap;
+  if (staged) {
+    const uint4* c4 = reinterpret_cast<const uint4*>(cand);
+    uint4* s4 = reinterpret_cast<uint4*>(cstage);
+    const uint32_t npairs = (cnt + 1u) >> 1;  // the buffer capacity is even: the pad pair is readable
+    for (uint32_t i = tid; i < npairs; i += THREADS) s4[i] = __ldcg(c4 + i);
+  }
+  __syncthreads();
+  // Visit (key, position) of every candidate -- or, on the exact fallback, of every position.
+  auto for_each = [&](auto&& fn) {
+    if (staged) {
+      for (uint32_t i = tid; i < cnt; i += THREADS) fn(cstage[2 * i], cstage[2 * i + 1]);
+    } else if (fast) {
+      // two candidates per 16-byte load, four loads in flight per thread
+      const uint4* c4 = reinterpret_cast<const uint4*>(cand);
+      const uint32_t npairs = cnt >> 1;
+      for (uint32_t i0 = tid; i0 < npairs; i0 += 4u * blockDim.x) {
+        uint4 e[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t i = i0 + k * blockDim.x;
+          if (i < npairs) e[k] = __ldcg(c4 + i);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (i0 + k * blockDim.x < npairs) {
+            fn(e[k].x, e[k].y);
+            fn(e[k].z, e[k].w);
+          }
+        }
+      }
+      if ((cnt & 1u) && tid == 0) {
+        const uint2 e = __ldcg(&cand[cnt - 1]);
+        fn(e.x, e.y);
+      }
+    } else {
+      for (int t = tid; t < n; t += blockDim.x) {
+        uint32_t w[RowGeom<R, FP8>::kWords];
+        load_row<R, FP8>(p, b, h, t, w);
+        fn(score_key(scale * row_dot<R, FP8>(w, u2)), (uint32_t)t);
+      }
+    }
+  };
+  constexpr int PER = kBins / THREADS;
+  // pass 0: top 11 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) { atomicAdd(&hist[k >> 21], 1u); });
+  __syncthreads();
+  uint32_t v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, (uint32_t)p.M, scan, digit);
+  const uint32_t d0 = digit[0];
+  uint32_t need = digit[1];
+  // pass 1: next 11 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) {
+    if ((k >> 21) == d0) atomicAdd(&hist[(k >> 10) & 0x7ffu], 1u);
+  });
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, need, scan, digit);
+  const uint32_t p22 = (d0 << 11) | digit[0];
+  need = digit[1];
+  // pass 2: last 10 bits
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
+  for_each([&](uint32_t k, uint32_t) {
+    if ((k >> 10) == p22) atomicAdd(&hist[k & 0x3ffu], 1u);
+  });
+  __syncthreads();
+  uint32_t v2[PER / 2];
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i) v2[i] = hist[tid * (PER / 2) + i];
+  find_digit(v2, need, scan, digit);
+  const uint32_t K = (p22 << 10) | digit[0];  // the M-th largest key
+  const uint32_t tie_take = digit[1];         // keys equal to K to keep, lowest positions first
+  for_each([&](uint32_t k, uint32_t pos) {
+    if (k > K)
+      atomicOr(&sel[pos >> 5], 1u << (pos & 31));
+    else if (k == K)
+      atomicOr(&tie[pos >> 5], 1u << (pos & 31));
+  });
+  __syncthreads();
+  // Keep the tie_take lowest tied positions; then emit every kept position in ascending order.
+  const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
+  const int wb = tid * wpt, we = min(nwords, wb + wpt);
+  uint32_t mine = 0;
+  for (int i = wb; i < we; ++i) mine += __popc(tie[i]);
+  uint32_t rank = block_exclusive_scan(mine, scan, nullptr);
+  for (int i = wb; i < we && rank < tie_take; ++i) {
+    uint32_t bits = tie[i];
+    while (bits && rank < tie_take) {
+      const uint32_t low = bits & (~bits + 1u);
+      sel[i] |= low;
+      bits ^= low;
+      ++rank;
+    }
+  }
+  mine = 0;
+  for (int i = wb; i < we; ++i) mine += __popc(sel[i]);
+  uint32_t slot = block_exclusive_scan(mine, scan, nullptr);
+  for (int i = wb; i < we; ++i) {
+    uint32_t bits = sel[i];
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      if (slot < (uint32_t)p.M) idx_out[slot] = i * 32 + bit;
+      ++slot;
+    }
+  }
+  if (tid == 0) p.count[bh] = p.M;
+}
+
+constexpr int kStreamChunk = 4096;        // positions per streaming CTA
+constexpr int kStreamStageBytes = 16384;  // projected-key bytes per pipeline stage
+constexpr int kStreamStages = 4;          // stages in the shared-memory ring of a streaming CTA
+
 template <int R, bool FP8>
-__global__ void __launch_bounds__(kIndexThreads, 2) lisa_index_stream_kernel(IndexParams p) {
-  __shared__ int32_t pages[kScoreChunk / 16];
+__global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(IndexParams p) {
+  extern __shared__ __align__(128) uint8_t ring[];  // kStreamStages x kStreamStageBytes
+  __shared__ const uint8_t* pbase[kStreamChunk / 16];  // global address of each page block of the chunk
   __shared__ uint32_t ckey[kStageCap];
   __shared__ uint32_t cpos[kStageCap];
   __shared__ uint32_t s_ncand, s_base;
   using Geo = RowGeom<R, FP8>;
-  constexpr int U = Geo::kUnroll;
+  constexpr int RB = Geo::kRowBytes;
+  constexpr int CPR = RB / 16;                 // 16-byte chunks per row
+  constexpr int RPS = kStreamStageBytes / RB;  // rows per stage
+  constexpr int RPT = RPS >= kIndexThreads ? RPS / kIndexThreads : 1;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * p.Hkv + h;
   const int n = load_seq_len(p, b);
   if (n <= p.M) return;
-  const int t_begin = blockIdx.x * kScoreChunk;
+  const int t_begin = blockIdx.x * kStreamChunk;
   if (t_begin >= n) return;
-  const int nrows = min(n - t_begin, kScoreChunk);
+  const int nrows = min(n - t_begin, kStreamChunk);
   if (tid == 0) s_ncand = 0u;
-  load_pages(p, b, t_begin >> p.log2ps, (nrows + p.ps - 1) >> p.log2ps, pages);
+  {
+    const int npg = (nrows + p.ps - 1) >> p.log2ps;
+    const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
+    for (int i = tid; i < npg; i += blockDim.x) {
+      int pid = p.page_table[(size_t)b * p.max_pages + (t_begin >> p.log2ps) + i];
+      if (pid < 0 || pid >= p.num_pages) {
+        flag_error(p.err, LISA_DEVERR_PAGE_ID);
+        pid = 0;
+      }
+      pbase[i] = base + ((((size_t)pid * p.Hkv + h) << p.log2ps) * RB);
+    }
+  }
   const uint32_t tau = p.tau[bh];
   const float scale = p.kproj_scale[h];
   float2 u2[R / 2];
   load_u2<R>(p.uq + bh * 32, u2);
   __syncthreads();
 
-  const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
-  for (int g0 = warp * U * 32; g0 < nrows; g0 += nwarps * U * 32) {
-    uint32_t w[U][Geo::kWords];
+  // Stage s holds rows [s * RPS, (s + 1) * RPS) of this chunk; the 16-byte chunks of a row are
+  // XOR-swizzled so that the row reads below are free of bank conflicts.  When a page block spans
+  // whole 512-byte segments, each warp copies segments (lane-contiguous, one page lookup per warp).
+  const bool seg_path = (p.ps * RB) % 512 == 0;
+  // this lane's 16-byte chunk inside a 512-byte segment: its row and swizzled destination offset
+  const int seg_row = (lane * 16) / RB, seg_part = ((lane * 16) % RB) / 16;
+  auto swz_off = [&](int r, int part) { return r * RB + ((part ^ (CPR > 1 ? ((r >> 2) & (CPR - 1)) : 0)) << 4); };
+  auto issue = [&](int stage, int slot) {
+    uint8_t* dst = ring + slot * kStreamStageBytes;
+    if (seg_path) {
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const int lr = g0 + k * 32 + lane;
-      if (lr < nrows) {
-        const int t = t_begin + lr;
-        const size_t row = (((size_t)pages[lr >> p.log2ps] * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1));
-        const uint8_t* src = base + row * Geo::kRowBytes;
+      for (int g = warp; g < kStreamStageBytes / 512; g += kIndexThreads / 32) {
+        const int r = g * (512 / RB) + seg_row;  // row within the stage
+        const int lr = stage * RPS + r;
+        const bool valid = lr < nrows;
+        const int vr = valid ? lr : 0;
+        const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + seg_part * 16;
+        cp_async_16(smem_u32(dst + swz_off(r, seg_part)), src, valid ? 16u : 0u);
+      }
+    } else {
 #pragma unroll
-        for (int l = 0; l < Geo::kLoads; ++l) load_vec<Geo::kVec>(src + l * Geo::kVec, &w[k][l * (Geo::kVec / 4)]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < Geo::kWords; ++i) w[k][i] = 0u;
+      for (int c = tid; c < kStreamStageBytes / 16; c += kIndexThreads) {
+        const int r = c / CPR, part = c % CPR;
+        const int lr = stage * RPS + r;
+        const bool valid = lr < nrows;
+        const int vr = valid ? lr : 0;
+        const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + part * 16;
+        cp_async_16(smem_u32(dst + swz_off(r, part)), src, valid ? 16u : 0u);
       }
     }
-    uint32_t key[U];
+  };
+  const int nstages = (nrows + RPS - 1) / RPS;
+#pragma unroll
+  for (int st = 0; st < kStreamStages - 1; ++st) {
+    if (st < nstages) issue(st, st);
+    cp_async_commit();
+  }
+  for (int st = 0; st < nstages; ++st) {
+    const int ns = st + kStreamStages - 1;
+    if (ns < nstages) issue(ns, ns % kStreamStages);
+    cp_async_commit();
+    cp_async_wait<kStreamStages - 1>();
+    __syncthreads();
+    const uint8_t* src = ring + (st % kStreamStages) * kStreamStageBytes;
+    uint32_t key[RPT];
     uint32_t mask = 0u;
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      key[k] = score_key(scale * row_dot<R, FP8>(w[k], u2));
-      if (g0 + k * 32 + lane < nrows && key[k] >= tau) mask |= 1u << k;
+    for (int k = 0; k < RPT; ++k) {
+      const int r = tid + k * kIndexThreads;
+      uint32_t w[Geo::kWords];
+#pragma unroll
+      for (int part = 0; part < CPR; ++part) {
+        const uint4 v = r < RPS ? *reinterpret_cast<const uint4*>(src + swz_off(r, part)) : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * part + 0] = v.x;
+        w[4 * part + 1] = v.y;
+        w[4 * part + 2] = v.z;
+        w[4 * part + 3] = v.w;
+      }
+      key[k] = score_key(scale * row_dot<R, FP8>(w, u2));
+      const int lr = st * RPS + r;
+      if (r < RPS && lr < nrows && key[k] >= tau) mask |= 1u << k;
     }
     if (__ballot_sync(0xffffffffu, mask != 0u)) {
       const uint32_t mine = __popc(mask);
@@ -426,31 +647,30 @@ __global__ void __launch_bounds__(kIndexThreads, 2) lisa_index_stream_kernel(Ind
       if (lane == 31) slot = atomicAdd(&s_ncand, incl);
       slot = __shfl_sync(0xffffffffu, slot, 31) + incl - mine;
 #pragma unroll
-      for (int k = 0; k < U; ++k) {
+      for (int k = 0; k < RPT; ++k) {
         if ((mask >> k) & 1u) {
           if (slot < (uint32_t)kStageCap) {
             ckey[slot] = key[k];
-            cpos[slot] = (uint32_t)(t_begin + g0 + k * 32 + lane);
+            cpos[slot] = (uint32_t)(t_begin + st * RPS + tid + k * kIndexThreads);
           }
           ++slot;
         }
       }
     }
+    __syncthreads();  // the slot is refilled by a later stage
   }
-  __syncthreads();
+  cp_async_wait<0>();
   const uint32_t nc = s_ncand;
   if (nc == 0u) return;
   if (tid == 0) s_base = atomicAdd(&p.ccount[bh], nc <= (uint32_t)kStageCap ? nc : (uint32_t)p.cap + 1u);
   __syncthreads();
-  if (nc > (uint32_t)kStageCap) return;  // the count now exceeds the capacity: finish recomputes
+  if (nc > (uint32_t)kStageCap) return;  // the count now exceeds the capacity: the exact path runs
   uint2* dst = reinterpret_cast<uint2*>(p.cand) + bh * (size_t)p.cap;
   for (uint32_t i = tid; i < nc; i += blockDim.x) {
     const uint32_t slot = s_base + i;
     if (slot < (uint32_t)p.cap) dst[slot] = make_uint2(ckey[i], cpos[i]);
   }
 }
-
-constexpr int kFinishThreads = 512;
 
 }  // namespace
 
@@ -684,132 +904,36 @@ __global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kIndexThr
 }
 
 
-size_t finish_smem_bytes(int max_seq_len) { return (size_t)2 * ((max_seq_len + 31) / 32) * 4; }
+constexpr int kFinishThreads = 512;
+constexpr uint32_t kFinishStageCap = 16384;  // candidates the finish kernel stages in shared memory
 
+__host__ __device__ static uint32_t finish_stage_cap(int cap) { return (uint32_t)cap < kFinishStageCap ? (uint32_t)cap : kFinishStageCap; }
+// Words of one position bitmap, rounded up to even so that the candidate stage is 16-byte aligned.
+__host__ __device__ static int finish_bitmap_words(int max_seq_len) { return ((max_seq_len + 63) / 64) * 2; }
+
+size_t finish_smem_bytes(int max_seq_len, int cap) {
+  return (size_t)2 * finish_bitmap_words(max_seq_len) * 4 + (size_t)finish_stage_cap(cap) * 8;
+}
+
+// One CTA per (KV head, sequence) with n > M: exact top-M from the streamed candidates.
 template <int R, bool FP8>
 __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(IndexParams p) {
   extern __shared__ __align__(16) uint32_t fsm[];
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t scan[32];
-  __shared__ uint32_t digit[2];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const size_t bh = (size_t)b * p.Hkv + h;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int n = load_seq_len(p, b);
-  int32_t* idx_out = p.idx + bh * p.M;
-  if (n <= p.M) {
-    for (int i = tid; i < p.M; i += blockDim.x) idx_out[i] = i < n ? i : -1;
-    if (tid == 0) p.count[bh] = n;
-    return;
-  }
-  const int nwords = (n + 31) >> 5;
-  uint32_t* sel = fsm;
-  uint32_t* tie = fsm + nwords;
-  for (int i = tid; i < nwords; i += blockDim.x) {
-    sel[i] = 0u;
-    tie[i] = 0u;
-  }
-  const uint32_t cnt = p.ccount[bh];
-  const bool fast = cnt >= (uint32_t)p.M && cnt <= (uint32_t)p.cap;
-  const uint2* cand = reinterpret_cast<const uint2*>(p.cand) + bh * (size_t)p.cap;
-  float2 u2[R / 2];
-  load_u2<R>(p.uq + bh * 32, u2);
-  const float scale = p.kproj_scale[h];
-  // Visit (key, position) of every candidate -- or, on the exact fallback, of every position.
-  auto for_each = [&](auto&& fn) {
-    if (fast) {
-      for (uint32_t i = tid; i < cnt; i += blockDim.x) {
-        const uint2 e = cand[i];
-        fn(e.x, e.y);
-      }
-    } else {
-      for (int t = tid; t < n; t += blockDim.x) {
-        uint32_t w[RowGeom<R, FP8>::kWords];
-        load_row<R, FP8>(p, b, h, t, w);
-        fn(score_key(scale * row_dot<R, FP8>(w, u2)), (uint32_t)t);
-      }
-    }
-  };
-  constexpr int PER = kBins / kFinishThreads;
-  // pass 0: top 11 bits
-  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
-  __syncthreads();
-  for_each([&](uint32_t k, uint32_t) { atomicAdd(&hist[k >> 21], 1u); });
-  __syncthreads();
-  uint32_t v[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
-  find_digit(v, (uint32_t)p.M, scan, digit);
-  const uint32_t d0 = digit[0];
-  uint32_t need = digit[1];
-  // pass 1: next 11 bits
-  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
-  __syncthreads();
-  for_each([&](uint32_t k, uint32_t) {
-    if ((k >> 21) == d0) atomicAdd(&hist[(k >> 10) & 0x7ffu], 1u);
-  });
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
-  find_digit(v, need, scan, digit);
-  const uint32_t p22 = (d0 << 11) | digit[0];
-  need = digit[1];
-  // pass 2: last 10 bits
-  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
-  __syncthreads();
-  for_each([&](uint32_t k, uint32_t) {
-    if ((k >> 10) == p22) atomicAdd(&hist[k & 0x3ffu], 1u);
-  });
-  __syncthreads();
-  uint32_t v2[PER / 2];
-#pragma unroll
-  for (int i = 0; i < PER / 2; ++i) v2[i] = hist[tid * (PER / 2) + i];
-  find_digit(v2, need, scan, digit);
-  const uint32_t K = (p22 << 10) | digit[0];  // the M-th largest key
-  const uint32_t tie_take = digit[1];         // keys equal to K to keep, lowest positions first
-  for_each([&](uint32_t k, uint32_t pos) {
-    if (k > K)
-      atomicOr(&sel[pos >> 5], 1u << (pos & 31));
-    else if (k == K)
-      atomicOr(&tie[pos >> 5], 1u << (pos & 31));
-  });
-  __syncthreads();
-  // Keep the tie_take lowest tied positions; then emit every kept position in ascending order.
-  const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
-  const int wb = tid * wpt, we = min(nwords, wb + wpt);
-  uint32_t mine = 0;
-  for (int i = wb; i < we; ++i) mine += __popc(tie[i]);
-  uint32_t rank = block_exclusive_scan(mine, scan, nullptr);
-  for (int i = wb; i < we && rank < tie_take; ++i) {
-    uint32_t bits = tie[i];
-    while (bits && rank < tie_take) {
-      const uint32_t low = bits & (~bits + 1u);
-      sel[i] |= low;
-      bits ^= low;
-      ++rank;
-    }
-  }
-  mine = 0;
-  for (int i = wb; i < we; ++i) mine += __popc(sel[i]);
-  uint32_t slot = block_exclusive_scan(mine, scan, nullptr);
-  for (int i = wb; i < we; ++i) {
-    uint32_t bits = sel[i];
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (slot < (uint32_t)p.M) idx_out[slot] = i * 32 + bit;
-      ++slot;
-    }
-  }
-  if (tid == 0) p.count[bh] = p.M;
+  if (n <= p.M) return;  // the sample kernel wrote the full set
+  uint32_t* cstage = fsm + 2 * finish_bitmap_words(p.max_seq_len);
+  finish_pair<R, FP8, kFinishThreads>(p, b, h, n, fsm, cstage, finish_stage_cap(p.cap));
 }
+
 
 // ---------------------------------------------------------------------------------------------
 // Host-side launchers (called from the C ABI layer after argument checks)
 // ---------------------------------------------------------------------------------------------
 
+// Opt in to the dynamic shared memory a launch uses (static + dynamic above 48 KB needs it).
 template <typename K>
 static cudaError_t set_smem(K kernel, size_t bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
@@ -827,15 +951,19 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream) {
   lisa_index_sample_kernel<R, FP8><<<dim3(p.Hkv, p.B), kSampleThreads, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const dim3 grid((p.max_seq_len + kScoreChunk - 1) / kScoreChunk, p.Hkv, p.B);
-  lisa_index_stream_kernel<R, FP8><<<grid, kIndexThreads, 0, stream>>>(p);
+  const dim3 grid((p.max_seq_len + kStreamChunk - 1) / kStreamChunk, p.Hkv, p.B);
+  const size_t ring = (size_t)kStreamStages * kStreamStageBytes;
+  auto k = lisa_index_stream_kernel<R, FP8>;
+  e = set_smem(k, ring);
+  if (e != cudaSuccess) return e;
+  k<<<grid, kIndexThreads, ring, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t smem = finish_smem_bytes(p.max_seq_len);
-  auto fk = lisa_index_finish_kernel<R, FP8>;
-  e = set_smem(fk, smem);
+  const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap);
+  auto f = lisa_index_finish_kernel<R, FP8>;
+  e = set_smem(f, fs);
   if (e != cudaSuccess) return e;
-  fk<<<dim3(p.Hkv, p.B), kFinishThreads, smem, stream>>>(p);
+  f<<<dim3(p.Hkv, p.B), kFinishThreads, fs, stream>>>(p);
   return cudaGetLastError();
 }
 

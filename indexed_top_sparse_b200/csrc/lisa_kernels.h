@@ -20,6 +20,8 @@ struct IndexParams {
   float* uq;           // [B][Hkv][32]: projected averaged query (written by the sample kernel)
   uint32_t* tau;       // [B][Hkv]: candidate threshold key
   uint32_t* ccount;    // [B][Hkv]: candidates appended (may exceed cap: overflow)
+  uint32_t* done;      // [B][Hkv]: streaming CTAs finished
+  uint32_t* acount;    // [B][Hkv]: attention partition counters, zeroed here for the fused path
   uint32_t* cand;      // [B][Hkv][cap][2]: (key, position)
   const int32_t* seq_lens;
   const int32_t* page_table;
@@ -46,17 +48,12 @@ struct AttnParams {
   const int32_t* count;
   float* o_part;   // [B][Hkv][splits][G][d], unnormalised, relative to the partition max
   float* ml_part;  // [B][Hkv][splits][G][2]: (max in log2 units, sum of 2^(x - max))
+  uint32_t* acount;  // [B][Hkv]: partitions finished (the last one merges and resets it to 0)
   uint32_t* err;
-};
-
-struct MergeParams {
-  int B, Hq, Hkv, d, splits;
-  const float* o_part;
-  const float* ml_part;
-  const __nv_bfloat16* q;
+  // Output of the merge (done by the last partition CTA of each (b, KV head)).
   __nv_bfloat16* out;
   float* lse;  // nullable
-  // linear branch (all null when absent)
+  // Optional linear branch (all null when absent).
   float* S;
   float* z;
   const __nv_bfloat16* k_new;
@@ -64,13 +61,13 @@ struct MergeParams {
   const float* gate;
 };
 
+
 size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
 cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream);
-size_t finish_smem_bytes(int max_seq_len);
+size_t finish_smem_bytes(int max_seq_len, int cap);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
-cudaError_t launch_merge(const MergeParams& p, cudaStream_t stream);
 
 }  // namespace lisa

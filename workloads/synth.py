@@ -346,11 +346,11 @@ def config2(device="cpu", seed=1002, **kw) -> DecodeProblem:
 
 
 def config3(device="cpu", seed=1003, **kw) -> DecodeProblem:
-    args = dict(B=16, Hq=64, Hkv=8, d=128, r=32, M=2048, n=131072)
+    args = dict(B=16, Hq=64, Hkv=8, d=128, r=32, M=2048, n=131072, paged=True)
     args.update(kw)
     n = args.pop("n")
     return make_problem(
-        name="config3", seq_lens=[n] * args["B"], page_size=64, paged=True, kproj_fp8=True,
+        name="config3", seq_lens=[n] * args["B"], page_size=64, kproj_fp8=True,
         plant=("cosine", 0.005), seed=seed, device=device, **args,
     )
 
