@@ -1,6 +1,8 @@
 """Build liblisa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m indexed_top_sparse_b200.build [--force] [--verbose]
+    python indexed_top_sparse_b200/build.py [--force] [--verbose]
+
+(run it as a script: importing the package loads the library this builds)
 
 The library links the CUDA runtime statically, so loading it needs no GPU;
 the first CUDA call does.
