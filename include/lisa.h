@@ -157,6 +157,22 @@ lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q,
                                     void* out, float* lse, void* ws, size_t ws_bytes,
                                     lisa_stream_t stream);
 
+/* Step 5 like lisa_sparse_decode_attn, for callers that cannot allocate device memory: it takes no
+ * workspace.  No counterpart on the pages: the write-ups do not discuss memory management.  Its
+ * scratch (partial sums of the attention partitions and their counters) is a fixed 8 MiB device
+ * array inside this library that every GPU which loads the library holds until the process exits;
+ * nothing is allocated or freed.  A desc whose scratch would exceed it -- about
+ * B * Hkv * lisa_num_splits(desc) * G * (d + 2) * 4 bytes plus small counters -- is rejected with
+ * LISA_ERR_WORKSPACE before anything is enqueued.  The first call on each device looks up the
+ * array's device address (a runtime call, done once per device); make that first call before any
+ * stream capture.  All calls share the one array, which keeps the last call's contents; each call
+ * clears its counters on `stream` first, and calls whose work overlaps on the GPU (other streams,
+ * other threads) race on it and must be serialised by the caller.  Device-side range checks still
+ * clamp bad indices, counts and page ids, but their flags are not reported by this entry point. */
+lisa_status lisa_sparse_decode_attn_noalloc(const lisa_decode_desc* desc, const void* q, const void* k_pool,
+                                            const void* v_pool, const int32_t* idx, const int32_t* count,
+                                            void* out, float* lse, lisa_stream_t stream);
+
 /* Steps 1-7 in one call.  reuse_idx/reuse_count (both or neither): take the index set from an
  * earlier layer and skip steps 1-4 (kproj_pool, P, kproj_scale may then be NULL).  idx_out/count_out
  * (both or neither, only without reuse): also return the index set.  lin may be NULL (no linear

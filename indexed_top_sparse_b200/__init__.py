@@ -25,6 +25,7 @@ from .binding import (  # noqa: F401
     lisa_index_topm,
     lisa_num_splits,
     lisa_sparse_decode_attn,
+    lisa_sparse_decode_attn_noalloc,
     lisa_status_string,
     lisa_topm_select,
     lisa_workspace_init,

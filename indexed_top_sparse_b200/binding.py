@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "liblisa.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m indexed_top_sparse_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python indexed_top_sparse_b200/build.py` "
         "(the library has no CPU fallback)"
     )
 _lib = ctypes.CDLL(LIB_PATH)
@@ -93,6 +93,7 @@ _sig = {
     "lisa_topm_select": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _S, _P]),
     "lisa_index_topm": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _I, _P, _P, _P, _P, _S, _P]),
     "lisa_sparse_decode_attn": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "lisa_sparse_decode_attn_noalloc": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _P, _P]),
     "lisa_fused_decode": (
         _I,
         [ctypes.POINTER(DecodeDesc), _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P,
@@ -203,6 +204,19 @@ def lisa_sparse_decode_attn(desc, q, k_pool, v_pool, idx, count, out, lse, ws, s
         _lib.lisa_sparse_decode_attn(ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(idx),
                                      _ptr(count), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
         "lisa_sparse_decode_attn",
+    )
+
+
+def lisa_sparse_decode_attn_noalloc(desc, q, k_pool, v_pool, idx, count, out, lse, stream=None) -> None:
+    """Attention over a given index set without a workspace (for callers that cannot allocate).
+
+    The library keeps the scratch in a fixed device array shared by all calls: calls must not overlap
+    on the GPU, and the first call on a device must come before any stream capture.
+    """
+    _check(
+        _lib.lisa_sparse_decode_attn_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(idx),
+                                             _ptr(count), _ptr(out), _ptr(lse), _stream(stream)),
+        "lisa_sparse_decode_attn_noalloc",
     )
 
 

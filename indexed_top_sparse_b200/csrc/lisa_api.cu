@@ -3,6 +3,8 @@
 
 #include <math.h>
 
+#include <mutex>
+
 #include "lisa.h"
 #include "lisa_common.cuh"
 #include "lisa_kernels.h"
@@ -210,6 +212,56 @@ lisa_status record(lisa_event_t ev, cudaStream_t stream) {
     if (_s != LISA_OK) return _s;       \
   } while (0)
 
+// ---------------------------------------------------------------------------------------------
+// Attention without a caller workspace, for callers that cannot allocate device memory (a
+// decode loop captured or scheduled by an engine that owns every allocation, or code that runs
+// where cudaMalloc is not allowed).  Its scratch -- error word, partition counters and the
+// split-attention partial sums -- is one file-scope device array of fixed size that every GPU
+// loading this library keeps until the process exits.
+// ---------------------------------------------------------------------------------------------
+
+constexpr size_t kNoAllocScratchBytes = (size_t)8 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device, looked up once per device.  In host
+// code the array's name stands for a host-side shadow, so the address must come from the runtime.
+lisa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LISA_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return LISA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      (void)cudaGetLastError();
+      return LISA_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return LISA_OK;
+}
+
+// Compact layout of the attention scratch inside the fixed array.
+Layout noalloc_layout(const lisa_decode_desc& d) {
+  Layout L = layout_of(d);
+  const size_t BH = (size_t)d.batch * d.num_kv_heads;
+  size_t off = kErrBytes;
+  L.off_acount = off;
+  off += align256(BH * 4);
+  L.off_opart = off;
+  off += align256(BH * (size_t)L.splits * L.G * (size_t)d.head_dim * 4);
+  L.off_ml = off;
+  off += align256(BH * (size_t)L.splits * L.G * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -309,6 +361,26 @@ lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q,
   LISA_TRY(clear_attn_counters(*desc, L, ws, st));
   return cuda_status(
       launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count, out, lse, nullptr), st));
+}
+
+lisa_status lisa_sparse_decode_attn_noalloc(const lisa_decode_desc* desc, const void* q, const void* k_pool,
+                                            const void* v_pool, const int32_t* idx, const int32_t* count,
+                                            void* out, float* lse, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || idx == nullptr || count == nullptr || out == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  const Layout L = noalloc_layout(*desc);
+  if (L.total > kNoAllocScratchBytes) return LISA_ERR_WORKSPACE;  // the fixed scratch is too small for desc
+  LISA_TRY(bind_device(out));
+  void* scratch = nullptr;
+  LISA_TRY(noalloc_scratch(&scratch));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // error word and partition counters start at zero on every call
+  LISA_TRY(cuda_status(cudaMemsetAsync(scratch, 0, L.off_opart, st)));
+  return cuda_status(
+      launch_sparse_attn(attn_params(*desc, L, scratch, q, k_pool, v_pool, idx, count, out, lse, nullptr), st));
 }
 
 lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,

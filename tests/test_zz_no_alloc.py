@@ -1,0 +1,58 @@
+"""Attention without a caller workspace, for callers that cannot allocate device memory.
+
+lisa_sparse_decode_attn_noalloc keeps its scratch in a fixed device array inside the library
+instead of a caller-provided workspace (useful to engines that own every allocation, or code that
+must not call cudaMalloc).  These checks compare it with lisa_sparse_decode_attn on the same index
+sets, over two calls in a row: the second call finds the first call's leftovers in the shared
+array and must not be affected by them.  This file is collected last on purpose.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import indexed_top_sparse_b200 as L
+from indexed_top_sparse_b200 import binding as Bnd
+from tests.parity import check_outputs
+from workloads import make_problem
+from workloads import run as R
+
+
+def _problem(dev, seed, **kw):
+    args = dict(name="noalloc", B=2, Hq=8, Hkv=2, d=128, r=32, M=512, seq_lens=[6000, 3001], page_size=64,
+                paged=True, kproj_fp8=True, plant=("cosine", 0.01), seed=seed)
+    args.update(kw)
+    return make_problem(device=dev, **args)
+
+
+@pytest.mark.gpu
+def test_noalloc_attention_matches_workspace_attention_on_two_calls(cuda_device):
+    probs = [
+        _problem(cuda_device, 301),
+        _problem(cuda_device, 302, B=8, Hq=32, Hkv=8, M=2048, seq_lens=[16384] * 8, paged=False),
+    ]
+    for prob in probs:  # two calls in a row through the no-allocation entry point
+        desc = R.desc_of(prob)
+        ws = R.workspace(prob, desc)
+        idx, count = R.index_topm(prob, ws, desc)
+        want_out, want_lse = R.attention(prob, idx, count, ws, desc)
+        out = torch.full_like(want_out, float("nan"))
+        lse = torch.full_like(want_lse, float("nan"))
+        L.lisa_sparse_decode_attn_noalloc(desc, prob.q, prob.k_pool, prob.v_pool, idx, count, out, lse)
+        torch.cuda.synchronize()
+        pairs = [(b, h) for b in range(prob.B) for h in range(prob.Hkv)]
+        check_outputs(out.float().cpu().double().numpy(), want_out.float().cpu().double().numpy(), pairs, prob.G)
+        assert np.allclose(lse.cpu().numpy(), want_lse.cpu().numpy(), rtol=1e-5, atol=1e-4)
+
+
+def test_noalloc_rejects_desc_beyond_its_fixed_scratch():
+    # 512 sequences x 8 KV heads x 16 partitions x 8 heads x 130 floats: far beyond the fixed 8 MiB
+    d = L.make_desc(batch=512, num_q_heads=64, num_kv_heads=8, head_dim=128, idx_dim=32, budget_m=16384,
+                    page_size=64, max_pages_per_seq=2048, max_seq_len=131072, num_pages=4096)
+    d.seq_lens = 0x1000
+    d.page_table = 0x2000
+    A = 0x1000
+    st = Bnd._lib.lisa_sparse_decode_attn_noalloc(ctypes.byref(d), A, A, A, A, A, A, None, None)
+    assert st == 3  # LISA_ERR_WORKSPACE, before anything touches the GPU
