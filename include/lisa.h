@@ -127,7 +127,9 @@ typedef struct {
 /* Workspace bytes any entry point needs for `desc` (0 if desc is invalid). Host only. */
 size_t lisa_workspace_size(const lisa_decode_desc* desc);
 
-/* Number of attention partitions per (b, KV head) the library uses for `desc` (0 if invalid). */
+/* Partial-result slots per (b, KV head) the attention step may use for `desc`: the stream-K grid
+ * splits the B * Hkv * ceil(M / 64) position tiles evenly over its CTAs, and each CTA writes one
+ * partial per (b, KV head) it touches (0 if desc is invalid). */
 int32_t lisa_num_splits(const lisa_decode_desc* desc);
 
 /* Zero the workspace error word (enqueued on stream). Call once after allocating ws. */

@@ -24,7 +24,7 @@ inline int ilog2(int x) {
 }
 
 struct Layout {
-  int G = 0, splits = 0, split_len = 0, chunk_max = 0, cap = 0;
+  int G = 0, grid = 0, tpp = 0, splits = 0, chunk_max = 0, cap = 0;  // splits: partial slots per pair
   size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0;
   size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_done = 0, off_acount = 0, off_cand = 0, total = 0;
 };
@@ -57,14 +57,15 @@ lisa_status check_idx_dim(const lisa_decode_desc* d) {
 Layout layout_of(const lisa_decode_desc& d) {
   Layout L;
   L.G = d.num_q_heads / d.num_kv_heads;
-  const int tiles = (d.budget_m + kAttnTile - 1) / kAttnTile;
-  const int pairs = d.batch > 0 ? d.batch * d.num_kv_heads : 1;
-  int splits = (kTargetAttnCtas + pairs - 1) / pairs;
-  const int min_splits = (d.budget_m + kMaxSplitLen - 1) / kMaxSplitLen;
-  if (splits < min_splits) splits = min_splits;
-  if (splits > tiles) splits = tiles;
-  L.split_len = ((tiles + splits - 1) / splits) * kAttnTile;
-  L.splits = (d.budget_m + L.split_len - 1) / L.split_len;
+  // Stream-K attention: kAttnGrid CTAs (at most one per tile) share the B * Hkv * ceil(M / 64) tiles
+  // evenly; a pair is covered by at most ceil(grid / pairs) + 1 CTAs, each writing one partial.
+  L.tpp = (d.budget_m + kAttnTile - 1) / kAttnTile;
+  const long long pairs = d.batch > 0 ? (long long)d.batch * d.num_kv_heads : 1;
+  const long long tiles = pairs * L.tpp;
+  long long grid = tiles < kAttnGrid ? tiles : kAttnGrid;
+  if (grid * kAttnMaxTiles < tiles) grid = (tiles + kAttnMaxTiles - 1) / kAttnMaxTiles;
+  L.grid = (int)grid;
+  L.splits = (int)((L.grid + pairs - 1) / pairs) + 1;
   const int per_cta = (d.max_seq_len + kClusterSize - 1) / kClusterSize;
   L.chunk_max = ((per_cta + d.page_size - 1) / d.page_size) * d.page_size;
   const size_t B = (size_t)d.batch, Hkv = (size_t)d.num_kv_heads;
@@ -165,8 +166,10 @@ AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, con
   p.max_pages = d.max_pages_per_seq;
   p.max_seq_len = d.max_seq_len;
   p.num_pages = d.num_pages;
-  p.splits = L.splits;
-  p.split_len = L.split_len;
+  p.npairs = d.batch * d.num_kv_heads;
+  p.tpp = L.tpp;
+  p.grid = L.grid;
+  p.max_seg = L.splits;
   const float scale = d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)d.head_dim);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.seq_lens = d.seq_lens;

@@ -4,20 +4,25 @@
 // decoding and on the specialised kernel): exact softmax attention of every query head over the
 // positions its KV head selected, using the original full-size bf16 keys and values read straight
 // from the paged cache -- no gathered copy -- with every head's own index set in one launch.  The
-// optional LISA linear branch and gate (LISA write-ups, "Архитектура LISA") are applied in the
-// merge kernel.
+// optional LISA linear branch and gate (LISA write-ups, "Архитектура LISA" / "Hybride architectuur
+// voor efficiëntie") are applied where the partitions of a (sequence, KV head) are merged.
 //
 // Design on B200:
-//  * Split-KV: a CTA owns (partition of the index list, KV head, sequence).  Row addresses of its
-//    positions are resolved once through the page table into shared memory; then 64-position tiles
-//    of K and V rows (256 B each at d = 128) are copied with 16-byte cp.async into a 3-stage ring
-//    (XOR-swizzled rows), so ~64 KB per CTA are in flight while the previous tile is consumed.
+//  * Stream-K over the flattened (sequence x KV head, 64-position tile) space: a fixed grid of
+//    CTAs, each taking an equal contiguous run of tiles, so every SM streams for the whole kernel
+//    with one pipeline fill, whatever the batch.  A CTA whose run crosses into the next
+//    (sequence, KV head) writes a partial (max, sum, unnormalised output) for the part it covered.
+//  * The CTA first resolves the pool rows of all its positions (at most kAttnMaxTiles tiles) through
+//    the page table, all index loads then all page loads in flight together; then 64 K rows and 64 V
+//    rows per tile (256 B each at d = 128) are copied with 16-byte cp.async into a 3-stage ring
+//    (XOR-swizzled), so two tiles are in flight while one is consumed.
 //  * The G query heads of one KV head are the n = 8 side of mma.m16n8k16 (bf16 in, fp32 accumulate):
 //    S^T = K Q^T with K rows from ldmatrix, then O^T += V^T P^T with V^T from ldmatrix.trans and P^T
-//    moved from the S^T accumulators by movmatrix.trans.  Tensor cores are used because the G-wide
-//    group makes this a real (if thin) contraction; the kernel stays bound by the row gathers.
-//  * Online softmax in base 2 per warp; warps merge in shared memory; partitions merge by
-//    log-sum-exp in the merge kernel, which also runs the linear branch and the gate.
+//    moved from the S^T accumulators by movmatrix.trans.  The G-wide group makes this a real, if
+//    thin, contraction; the kernel stays bound by the row gathers.
+//  * Online softmax in base 2 per warp; the four warps merge in shared memory; the partials of a
+//    (sequence, KV head) are merged by log-sum-exp in the CTA that writes the last of them (a fenced
+//    atomic counter, no waiting), which also runs the linear branch and the gate.
 
 #include "lisa_common.cuh"
 #include "lisa_kernels.h"
@@ -28,6 +33,7 @@ namespace {
 
 #define kNegInf (__int_as_float(0xff800000u))
 
+
 template <int D>
 struct AttnGeom {
   static constexpr int kRowBytes = D * 2;
@@ -35,11 +41,16 @@ struct AttnGeom {
   static constexpr int kTileBytes = kAttnTile * kRowBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;  // K tile then V tile
   static constexpr int kRowsPerPass = kAttnThreads / kChunks;
-  static constexpr size_t kSmem = (size_t)kAttnStages * kStageBytes + (size_t)kMaxSplitLen * 4;
+  static constexpr size_t kSmem = (size_t)kAttnStages * kStageBytes + (size_t)kAttnMaxTiles * kAttnTile * 4;
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk, int row_bytes) {
   return (uint32_t)(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+}
+
+// CTA (of `grid`) whose tile run contains flattened tile x of `total`: run c is [c*T/C, (c+1)*T/C).
+__device__ __forceinline__ int owner_cta(long long x, long long total, int grid) {
+  return (int)(((x + 1) * grid + total - 1) / total) - 1;
 }
 
 }  // namespace
@@ -48,54 +59,53 @@ size_t attn_smem_bytes(int d) { return d == 64 ? AttnGeom<64>::kSmem : AttnGeom<
 
 __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
-// Merge the partitions of one (b, KV head) for its G query heads; optional linear branch + gate.
-// Run by the 128 threads of the last partition CTA of (b, h); thread e owns output column e.
+// Merge the nseg partials of one (b, KV head) for its G query heads; optional linear branch + gate.
+// Run by the 128 threads of the CTA that wrote the last partial; thread e owns output column e.
 template <int D>
-__device__ void merge_pair(const AttnParams& p, int b, int h) {
+__device__ void merge_pair(const AttnParams& p, int b, int h, int nseg) {
   __shared__ float fk[D];
   __shared__ float fq[kMaxG][D];
   __shared__ float zn[D];
   __shared__ float den[kMaxG];
-  __shared__ float wsplit[kMaxG][64];
+  __shared__ float wseg[kMaxG][64];
   __shared__ float mstar[kMaxG], lstar[kMaxG];
   const int G = p.Hq / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = (size_t)b * p.Hkv + h;
-  const float* mlp = p.ml_part + bh * p.splits * G * 2;
-  const float* op = p.o_part + bh * p.splits * G * D;
+  const float* mlp = p.ml_part + bh * p.max_seg * G * 2;
+  const float* op = p.o_part + bh * p.max_seg * G * D;
 
-  // Partition weights, in chunks of 64 partitions.
   float acc[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
   if (tid < G) {
     float mx = kNegInf;
-    for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, __ldcg(&mlp[(s * G + tid) * 2]));
+    for (int s = 0; s < nseg; ++s) mx = fmaxf(mx, __ldcg(&mlp[(s * G + tid) * 2]));
     float l = 0.f;
     if (mx != kNegInf)
-      for (int s = 0; s < p.splits; ++s) {
+      for (int s = 0; s < nseg; ++s) {
         const float ms = __ldcg(&mlp[(s * G + tid) * 2]);
         if (ms != kNegInf) l += __ldcg(&mlp[(s * G + tid) * 2 + 1]) * exp2f(ms - mx);
       }
     mstar[tid] = mx;
     lstar[tid] = l;
   }
-  for (int s0 = 0; s0 < p.splits; s0 += 64) {
+  for (int s0 = 0; s0 < nseg; s0 += 64) {
     __syncthreads();
     for (int e = tid; e < G * 64; e += blockDim.x) {
       const int g = e / 64, s = s0 + (e - g * 64);
       float w = 0.f;
-      if (s < p.splits) {
+      if (s < nseg) {
         const float ms = __ldcg(&mlp[(s * G + g) * 2]);
         if (ms != kNegInf && mstar[g] != kNegInf) w = exp2f(ms - mstar[g]);
       }
-      wsplit[g][e - g * 64] = w;
+      wseg[g][e - g * 64] = w;
     }
     __syncthreads();
     if (tid < D) {
-      const int s1 = min(p.splits, s0 + 64);
+      const int s1 = min(nseg, s0 + 64);
       for (int s = s0; s < s1; ++s)
-        for (int g = 0; g < G; ++g) acc[g] += wsplit[g][s - s0] * __ldcg(&op[((size_t)s * G + g) * D + tid]);
+        for (int g = 0; g < G; ++g) acc[g] += wseg[g][s - s0] * __ldcg(&op[((size_t)s * G + g) * D + tid]);
     }
   }
   float sparse[kMaxG];
@@ -156,118 +166,241 @@ __device__ void merge_pair(const AttnParams& p, int b, int h) {
   }
 }
 
+// Valid positions of (b, h): count clamped to [0, min(M, n_b)] (flagging out-of-range values).
+__device__ __forceinline__ int pair_count(const AttnParams& p, int pr, int b, bool flag) {
+  int n = p.seq_lens[b];
+  if (n < 0 || n > p.max_seq_len) {
+    if (flag) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
+    n = n < 0 ? 0 : p.max_seq_len;
+  }
+  const int limit = min(p.M, n);
+  int cnt = p.count[pr];
+  if (cnt < 0 || cnt > limit) {
+    if (flag) flag_error(p.err, LISA_DEVERR_COUNT);
+    cnt = cnt < 0 ? 0 : limit;
+  }
+  return cnt;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnParams p) {
   using Geo = AttnGeom<D>;
   extern __shared__ __align__(128) uint8_t smem[];
-  uint32_t* rows = reinterpret_cast<uint32_t*>(smem + kAttnStages * Geo::kStageBytes);
+  uint32_t* rows_sm = reinterpret_cast<uint32_t*>(smem + kAttnStages * Geo::kStageBytes);  // [tile][64]
+  __shared__ uint32_t s_last;
 
-  const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int G = p.Hq / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g_ = lane >> 2, t_ = lane & 3;
-
-  int n = p.seq_lens[b];
-  if (n < 0 || n > p.max_seq_len) {
-    if (s == 0 && tid == 0) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
-    n = n < 0 ? 0 : p.max_seq_len;
-  }
-  const int limit = min(p.M, n);
-  int cnt = p.count[(size_t)b * p.Hkv + h];
-  if (cnt < 0 || cnt > limit) {
-    if (s == 0 && tid == 0) flag_error(p.err, LISA_DEVERR_COUNT);
-    cnt = cnt < 0 ? 0 : limit;
-  }
-  const int p0 = s * p.split_len;
-  const int len = max(0, min(cnt, p0 + p.split_len) - p0);
-
-  // Resolve the partition's positions to pool rows (row = (page * ps + slot) * Hkv + h).
-  const int32_t* idxp = p.idx + ((size_t)b * p.Hkv + h) * p.M + p0;
-  const int32_t* table = p.page_table + (size_t)b * p.max_pages;
-  for (int i = tid; i < len; i += kAttnThreads) {
-    int t = idxp[i];
-    if (t < 0 || t >= n) {
-      flag_error(p.err, LISA_DEVERR_INDEX);
-      t = 0;
-    }
-    int pg = table[t >> p.log2ps];
-    if (pg < 0 || pg >= p.num_pages) {
-      flag_error(p.err, LISA_DEVERR_PAGE_ID);
-      pg = 0;
-    }
-    rows[i] = ((uint32_t)pg * (uint32_t)p.ps + (uint32_t)(t & (p.ps - 1))) * (uint32_t)p.Hkv + (uint32_t)h;
-  }
-
-  // Q^T fragments (B operand, k = d, n = query head of the group); heads >= G are zero.
-  uint32_t qf[D / 16][2];
-  {
-    const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)h * G + (g_ < G ? g_ : 0)) * D;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      qf[kk][0] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_) : 0u;
-      qf[kk][1] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_ + 8) : 0u;
-    }
-  }
-  __syncthreads();
-
-  const int ntiles = (len + kAttnTile - 1) / kAttnTile;
+  const int C = gridDim.x, c = blockIdx.x;
+  const long long T = (long long)p.npairs * p.tpp;
+  const int t_lo = (int)((long long)c * T / C), t_hi = (int)((long long)(c + 1) * T / C);
+  const int ntile = t_hi - t_lo;
   const uint8_t* kbase = reinterpret_cast<const uint8_t*>(p.k_pool);
   const uint8_t* vbase = reinterpret_cast<const uint8_t*>(p.v_pool);
-  auto issue = [&](int tile, int stage) {
-    uint8_t* kdst = smem + stage * Geo::kStageBytes;
+  constexpr uint32_t kNoRow = 0xffffffffu;
+
+  // Pool rows (row = (page * ps + slot) * Hkv + h) of every position of this CTA's tiles, or kNoRow
+  // past the pair's count: all index loads are issued first, then all page-table loads.
+  {
+    constexpr int kPer = kAttnMaxTiles * kAttnTile / kAttnThreads;
+    int tpos[kPer];
+    uint32_t meta[kPer];  // pair-local validity and (b, h) of each slot
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int e = tid + k * kAttnThreads, i = e / kAttnTile;
+      tpos[k] = -1;
+      meta[k] = 0u;
+      if (i < ntile) {
+        const int gt = t_lo + i, pr = gt / p.tpp, lt = gt - pr * p.tpp;
+        const int b = pr / p.Hkv;
+        const int cnt = pair_count(p, pr, b, (e % kAttnTile) == 0 && lt == 0);
+        const int pos = lt * kAttnTile + (e % kAttnTile);
+        if (pos < cnt) {
+          tpos[k] = p.idx[(size_t)pr * p.M + pos];
+          meta[k] = 1u;
+        }
+      }
+    }
+    int pgs[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int e = tid + k * kAttnThreads, i = e / kAttnTile;
+      pgs[k] = 0;
+      if (meta[k]) {
+        const int gt = t_lo + i, pr = gt / p.tpp, b = pr / p.Hkv;
+        const int n = min(max(p.seq_lens[b], 0), p.max_seq_len);
+        if (tpos[k] < 0 || tpos[k] >= n) {
+          flag_error(p.err, LISA_DEVERR_INDEX);
+          tpos[k] = 0;
+        }
+        pgs[k] = p.page_table[(size_t)b * p.max_pages + (tpos[k] >> p.log2ps)];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int e = tid + k * kAttnThreads, i = e / kAttnTile;
+      if (i < ntile) {
+        uint32_t row = kNoRow;
+        if (meta[k]) {
+          const int gt = t_lo + i, pr = gt / p.tpp, h = pr % p.Hkv;
+          int pg = pgs[k];
+          if (pg < 0 || pg >= p.num_pages) {
+            flag_error(p.err, LISA_DEVERR_PAGE_ID);
+            pg = 0;
+          }
+          row = ((uint32_t)pg * (uint32_t)p.ps + (uint32_t)(tpos[k] & (p.ps - 1))) * (uint32_t)p.Hkv + (uint32_t)h;
+        }
+        rows_sm[e] = row;
+      }
+    }
+  }
+  // 16-byte cp.async copies of tile i's K and V rows into stage i % kAttnStages (zeros past the count).
+  auto issue = [&](int i) {
+    if (i >= ntile) return;
+    uint8_t* kdst = smem + (i % kAttnStages) * Geo::kStageBytes;
     uint8_t* vdst = kdst + Geo::kTileBytes;
-    const int c = tid % Geo::kChunks;
+    const uint32_t* rows = rows_sm + i * kAttnTile;
+    const int ch = tid % Geo::kChunks;
 #pragma unroll
     for (int r = tid / Geo::kChunks; r < kAttnTile; r += Geo::kRowsPerPass) {
-      const int li = tile * kAttnTile + r;
-      const bool valid = li < len;
-      const size_t off = (size_t)(valid ? rows[li] : 0u) * Geo::kRowBytes + (size_t)c * 16;
-      const uint32_t so = swz(r, c, Geo::kRowBytes);
+      const uint32_t row = rows[r];
+      const bool valid = row != kNoRow;
+      const size_t off = (size_t)(valid ? row : 0u) * Geo::kRowBytes + (size_t)ch * 16;
+      const uint32_t so = swz(r, ch, Geo::kRowBytes);
       cp_async_16(smem_u32(kdst + so), kbase + off, valid ? 16u : 0u);
       cp_async_16(smem_u32(vdst + so), vbase + off, valid ? 16u : 0u);
     }
   };
 
+  __syncthreads();
 #pragma unroll
   for (int st = 0; st < kAttnStages - 1; ++st) {
-    if (st < ntiles) issue(st, st);
+    issue(st);
     cp_async_commit();
   }
 
-  float m_run[2] = {kNegInf, kNegInf};  // per head 2t_, 2t_+1 (log2 units)
-  float l_run[2] = {0.f, 0.f};          // partial over this lane's rows
+  float m_run[2], l_run[2];  // per head 2t_, 2t_+1 (log2 units); l is a partial over this lane's rows
   float o[D / 16][4];
+  uint32_t qf[D / 16][2];  // Q^T fragments (B operand, k = d, n = query head of the group)
+  int cur = -1, cur_cnt = 0;
+
+  // Write the CTA's partial for pair pr (its warps merged in shared memory at `scratch`) and, if it
+  // is the last of the pair's partials, merge them into the output.
+  auto flush = [&](int pr, uint8_t* scratch) {
+    const int b = pr / p.Hkv, h = pr - b * p.Hkv;
 #pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+    for (int off = 4; off < 32; off <<= 1) {
+      l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+      l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+    }
+    float* obuf = reinterpret_cast<float*>(scratch);  // [warp][head][D]
+    float* wm = obuf + 4 * kMaxG * D;
+    float* wl = wm + 4 * kMaxG;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      const int d0 = 16 * mt + g_;
+      obuf[(warp * kMaxG + 2 * t_) * D + d0] = o[mt][0];
+      obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0] = o[mt][1];
+      obuf[(warp * kMaxG + 2 * t_) * D + d0 + 8] = o[mt][2];
+      obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0 + 8] = o[mt][3];
+    }
+    if (g_ == 0) {
+      wm[warp * kMaxG + 2 * t_] = m_run[0];
+      wm[warp * kMaxG + 2 * t_ + 1] = m_run[1];
+      wl[warp * kMaxG + 2 * t_] = l_run[0];
+      wl[warp * kMaxG + 2 * t_ + 1] = l_run[1];
+    }
+    __syncthreads();
+    const long long first = (long long)pr * p.tpp;
+    const int c_first = owner_cta(first, T, C);
+    const int nseg = owner_cta(first + p.tpp - 1, T, C) - c_first + 1;
+    const size_t part = (size_t)pr * p.max_seg + (c - c_first);
+    float* op = p.o_part + part * G * D;
+    for (int e = tid; e < G * D; e += kAttnThreads) {
+      const int gg = e / D, dd = e - gg * D;
+      float mx = kNegInf;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + gg]);
+      float acc = 0.f;
+      if (mx != kNegInf) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float mw = wm[w * kMaxG + gg];
+          if (mw != kNegInf) acc += obuf[(w * kMaxG + gg) * D + dd] * exp2f(mw - mx);
+        }
+      }
+      op[e] = acc;
+    }
+    if (tid < G) {
+      float mx = kNegInf;
+      for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + tid]);
+      float l = 0.f;
+      if (mx != kNegInf) {
+        for (int w = 0; w < 4; ++w) {
+          const float mw = wm[w * kMaxG + tid];
+          if (mw != kNegInf) l += wl[w * kMaxG + tid] * exp2f(mw - mx);
+        }
+      }
+      p.ml_part[(part * G + tid) * 2 + 0] = mx;
+      p.ml_part[(part * G + tid) * 2 + 1] = l;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+      s_last = atomicAdd(&p.acount[pr], 1u) == (uint32_t)nseg - 1u;
+      if (s_last) p.acount[pr] = 0u;
+    }
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      merge_pair<D>(p, b, h, nseg);
+    }
+    __syncthreads();  // the scratch stage is refilled next
+  };
 
   const int rbase = warp * 16;
-  for (int tile = 0; tile < ntiles; ++tile) {
-    const int nt = tile + kAttnStages - 1;
-    if (nt < ntiles) issue(nt, nt % kAttnStages);
+  for (int i = 0; i < ntile; ++i) {
+    const int gt = t_lo + i, pr = gt / p.tpp, lt = gt - pr * p.tpp;
+    if (pr != cur) {
+      if (cur >= 0) flush(cur, smem + ((i + kAttnStages - 1) % kAttnStages) * Geo::kStageBytes);
+      cur = pr;
+      const int b = pr / p.Hkv, h = pr - b * p.Hkv;
+      cur_cnt = pair_count(p, pr, b, false);
+      const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)h * G + (g_ < G ? g_ : 0)) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qf[kk][0] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_) : 0u;
+        qf[kk][1] = g_ < G ? *reinterpret_cast<const uint32_t*>(qrow + 16 * kk + 2 * t_ + 8) : 0u;
+      }
+      m_run[0] = m_run[1] = kNegInf;
+      l_run[0] = l_run[1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+    }
+    issue(i + kAttnStages - 1);
     cp_async_commit();
     cp_async_wait<kAttnStages - 1>();
     __syncthreads();
 
-    const uint8_t* ks = smem + (tile % kAttnStages) * Geo::kStageBytes;
+    const uint8_t* ks = smem + (i % kAttnStages) * Geo::kStageBytes;
     const uint8_t* vs = ks + Geo::kTileBytes;
-
     // S^T (16 positions x 8 heads) = K_tile(16 x D) . Q^T(D x 8)
     float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int r = rbase + (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int c = 2 * kk + (lane >> 4);
+      const int cc = 2 * kk + (lane >> 4);
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(smem_u32(ks + swz(r, c, Geo::kRowBytes)), a0, a1, a2, a3);
+      ldmatrix_x4(smem_u32(ks + swz(r, cc, Geo::kRowBytes)), a0, a1, a2, a3);
       mma_bf16_16816(sacc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
     }
-
     // Online softmax (base 2).  c0,c1: position rbase+g_, heads 2t_,2t_+1; c2,c3: position +8.
-    const int pos0 = tile * kAttnTile + rbase + g_;
+    const int pos0 = lt * kAttnTile + rbase + g_;
     float x00 = sacc[0] * p.scale_log2, x01 = sacc[1] * p.scale_log2;
     float x10 = sacc[2] * p.scale_log2, x11 = sacc[3] * p.scale_log2;
-    if (pos0 >= len) x00 = x01 = kNegInf;
-    if (pos0 + 8 >= len) x10 = x11 = kNegInf;
+    if (pos0 >= cur_cnt) x00 = x01 = kNegInf;
+    if (pos0 + 8 >= cur_cnt) x10 = x11 = kNegInf;
     float mA = fmaxf(x00, x10), mB = fmaxf(x01, x11);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
@@ -295,107 +428,34 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     // P^T (16 positions x 8 heads) in bf16 -> B fragments of the PV product via an 8x8 transpose.
     const uint32_t pb0 = movmatrix_trans(pack_bf16x2(pA0, pB0));
     const uint32_t pb1 = movmatrix_trans(pack_bf16x2(pA1, pB1));
-
     // O^T (D x 8) += V^T(D x 16 positions) . P^T(16 x 8)
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
       const int r = rbase + (lane & 7) + ((lane >> 4) & 1) * 8;
-      const int c = 2 * mt + ((lane >> 3) & 1);
+      const int cc = 2 * mt + ((lane >> 3) & 1);
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4_trans(smem_u32(vs + swz(r, c, Geo::kRowBytes)), a0, a1, a2, a3);
+      ldmatrix_x4_trans(smem_u32(vs + swz(r, cc, Geo::kRowBytes)), a0, a1, a2, a3);
       mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
     }
     __syncthreads();  // the stage is refilled by a later iteration
   }
   cp_async_wait<0>();
-
-  // Reduce the lane-partial sums over the 8 row groups.
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
-    l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
-  }
-  __syncthreads();
-  // Per-warp results to shared memory: obuf[warp][head][D], wm/wl[warp][head].
-  float* obuf = reinterpret_cast<float*>(smem);
-  float* wm = obuf + 4 * kMaxG * D;
-  float* wl = wm + 4 * kMaxG;
-#pragma unroll
-  for (int mt = 0; mt < D / 16; ++mt) {
-    const int d0 = 16 * mt + g_;
-    obuf[(warp * kMaxG + 2 * t_) * D + d0] = o[mt][0];
-    obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0] = o[mt][1];
-    obuf[(warp * kMaxG + 2 * t_) * D + d0 + 8] = o[mt][2];
-    obuf[(warp * kMaxG + 2 * t_ + 1) * D + d0 + 8] = o[mt][3];
-  }
-  if (g_ == 0) {
-    wm[warp * kMaxG + 2 * t_] = m_run[0];
-    wm[warp * kMaxG + 2 * t_ + 1] = m_run[1];
-    wl[warp * kMaxG + 2 * t_] = l_run[0];
-    wl[warp * kMaxG + 2 * t_ + 1] = l_run[1];
-  }
-  __syncthreads();
-  const size_t part = ((size_t)b * p.Hkv + h) * p.splits + s;
-  float* op = p.o_part + part * G * D;
-  for (int e = tid; e < G * D; e += kAttnThreads) {
-    const int gg = e / D, dd = e - gg * D;
-    float mx = kNegInf;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + gg]);
-    float acc = 0.f;
-    if (mx != kNegInf) {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float mw = wm[w * kMaxG + gg];
-        if (mw != kNegInf) acc += obuf[(w * kMaxG + gg) * D + dd] * exp2f(mw - mx);
-      }
-    }
-    op[e] = acc;
-  }
-  if (tid < G) {
-    float mx = kNegInf;
-    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, wm[w * kMaxG + tid]);
-    float l = 0.f;
-    if (mx != kNegInf) {
-      for (int w = 0; w < 4; ++w) {
-        const float mw = wm[w * kMaxG + tid];
-        if (mw != kNegInf) l += wl[w * kMaxG + tid] * exp2f(mw - mx);
-      }
-    }
-    p.ml_part[(part * G + tid) * 2 + 0] = mx;
-    p.ml_part[(part * G + tid) * 2 + 1] = l;
-  }
-  // The CTA that completes the last partition of (b, h) merges them (no waiting on other CTAs).
-  __shared__ uint32_t s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const size_t bh = (size_t)b * p.Hkv + h;
-    s_last = atomicAdd(&p.acount[bh], 1u) == (uint32_t)p.splits - 1u;
-    if (s_last) p.acount[bh] = 0u;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    merge_pair<D>(p, b, h);
-  }
+  if (cur >= 0) flush(cur, smem + ((ntile - 1) % kAttnStages) * Geo::kStageBytes);
 }
 
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream) {
-  dim3 grid(p.splits, p.Hkv, p.B);
   if (p.d == 64) {
     auto k = lisa_sparse_attn_kernel<64>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<64>::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kAttnThreads, AttnGeom<64>::kSmem, stream>>>(p);
+    k<<<p.grid, kAttnThreads, AttnGeom<64>::kSmem, stream>>>(p);
   } else {
     auto k = lisa_sparse_attn_kernel<128>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<128>::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kAttnThreads, AttnGeom<128>::kSmem, stream>>>(p);
+    k<<<p.grid, kAttnThreads, AttnGeom<128>::kSmem, stream>>>(p);
   }
   return cudaGetLastError();
 }
-
 
 }  // namespace lisa

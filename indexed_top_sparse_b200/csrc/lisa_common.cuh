@@ -17,7 +17,8 @@ constexpr int kBins = 2048;           // radix digits per pass (11 bits)
 constexpr int kAttnThreads = 128;     // threads of an attention CTA (4 warps)
 constexpr int kAttnTile = 64;         // positions per pipeline stage (16 per warp)
 constexpr int kAttnStages = 3;        // cp.async pipeline depth
-constexpr int kMaxSplitLen = 1024;    // positions per attention partition, at most
+constexpr int kAttnGrid = 2 * 148;    // stream-K attention CTAs: two per B200 SM (more if needed)
+constexpr int kAttnMaxTiles = 16;     // 64-position tiles per attention CTA, at most
 constexpr int kMaxG = 8;              // query heads per KV head (mma n = 8)
 constexpr int kMaxSeqLen = 262144;
 constexpr int kMaxBudget = 16384;

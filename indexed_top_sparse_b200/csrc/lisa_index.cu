@@ -65,9 +65,15 @@ __device__ __forceinline__ void ffma2(float2& c, float2 a, float2 b) {
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
 }
 
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t two_bytes) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_bytes, __NV_E4M3);
-  return __half22float2(*reinterpret_cast<__half2*>(&h));
+// Four E4M3 values packed in a word -> four floats (hardware e4m3x2 -> f16x2, then f16 -> f32).
+__device__ __forceinline__ void e4m3x4_to_float(uint32_t w, float2& lo, float2& hi) {
+  asm("{\n\t.reg .b16 b0, b1, h0, h1, h2, h3;\n\t.reg .b32 p0, p1;\n\t"
+      "mov.b32 {b0, b1}, %4;\n\t"
+      "cvt.rn.f16x2.e4m3x2 p0, b0;\n\tcvt.rn.f16x2.e4m3x2 p1, b1;\n\t"
+      "mov.b32 {h0, h1}, p0;\n\tmov.b32 {h2, h3}, p1;\n\t"
+      "cvt.f32.f16 %0, h0;\n\tcvt.f32.f16 %1, h1;\n\tcvt.f32.f16 %2, h2;\n\tcvt.f32.f16 %3, h3;\n\t}\n"
+      : "=f"(lo.x), "=f"(lo.y), "=f"(hi.x), "=f"(hi.y)
+      : "r"(w));
 }
 
 // <u, row> for one row held in registers (element e of the row pairs with u[e]).
@@ -77,8 +83,10 @@ __device__ __forceinline__ float row_dot(const uint32_t* w, const float2* u2) {
   if constexpr (FP8) {
 #pragma unroll
     for (int i = 0; i < R / 4; ++i) {
-      ffma2(a0, e4m3x2_to_float2(w[i] & 0xffffu), u2[2 * i]);
-      ffma2(a1, e4m3x2_to_float2(w[i] >> 16), u2[2 * i + 1]);
+      float2 lo, hi;
+      e4m3x4_to_float(w[i], lo, hi);
+      ffma2(a0, lo, u2[2 * i]);
+      ffma2(a1, hi, u2[2 * i + 1]);
     }
   } else {
 #pragma unroll
@@ -530,22 +538,28 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
   if (tid == 0) p.count[bh] = p.M;
 }
 
-constexpr int kStreamChunk = 4096;        // positions per streaming CTA
-constexpr int kStreamStageBytes = 16384;  // projected-key bytes per pipeline stage
-constexpr int kStreamStages = 4;          // stages in the shared-memory ring of a streaming CTA
+constexpr int kStreamChunk = 4096;        // positions per streaming CTA (kStreamChunk / 8 per warp)
+constexpr int kStreamStageBytes = 2048;   // projected-key bytes per warp pipeline stage
+constexpr int kStreamStages = 4;          // stages in each warp's shared-memory ring
 
+// Each warp streams its own contiguous eighth of the CTA's chunk through a private cp.async ring:
+// a lane waits only for its own copies and the warp synchronises with __syncwarp, so the streaming
+// loop has no CTA-wide barrier.  Stage s of a warp holds rows [s * RPS, (s + 1) * RPS) of its range
+// (16-byte chunks XOR-swizzled within each row so that the row reads are free of bank conflicts).
 template <int R, bool FP8>
 __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(IndexParams p) {
-  extern __shared__ __align__(128) uint8_t ring[];  // kStreamStages x kStreamStageBytes
+  extern __shared__ __align__(128) uint8_t ring[];  // [warp][kStreamStages][kStreamStageBytes]
   __shared__ const uint8_t* pbase[kStreamChunk / 16];  // global address of each page block of the chunk
   __shared__ uint32_t ckey[kStageCap];
   __shared__ uint32_t cpos[kStageCap];
   __shared__ uint32_t s_ncand, s_base;
   using Geo = RowGeom<R, FP8>;
   constexpr int RB = Geo::kRowBytes;
-  constexpr int CPR = RB / 16;                 // 16-byte chunks per row
-  constexpr int RPS = kStreamStageBytes / RB;  // rows per stage
-  constexpr int RPT = RPS >= kIndexThreads ? RPS / kIndexThreads : 1;
+  constexpr int CPR = RB / 16;                            // 16-byte chunks per row
+  constexpr int RPS = kStreamStageBytes / RB;             // rows per stage
+  constexpr int RPL = RPS >= 32 ? RPS / 32 : 1;           // rows per lane per stage
+  constexpr int WARPS = kIndexThreads / 32;
+  constexpr int WROWS = kStreamChunk / WARPS;             // rows per warp
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * p.Hkv + h;
@@ -573,55 +587,41 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
   load_u2<R>(p.uq + bh * 32, u2);
   __syncthreads();
 
-  // Stage s holds rows [s * RPS, (s + 1) * RPS) of this chunk; the 16-byte chunks of a row are
-  // XOR-swizzled so that the row reads below are free of bank conflicts.  When a page block spans
-  // whole 512-byte segments, each warp copies segments (lane-contiguous, one page lookup per warp).
-  const bool seg_path = (p.ps * RB) % 512 == 0;
-  // this lane's 16-byte chunk inside a 512-byte segment: its row and swizzled destination offset
-  const int seg_row = (lane * 16) / RB, seg_part = ((lane * 16) % RB) / 16;
+  uint8_t* wring = ring + warp * (kStreamStages * kStreamStageBytes);
+  const int w0 = warp * WROWS;                               // first row of this warp (chunk-relative)
+  const int wrows = max(0, min(nrows - w0, WROWS));          // rows this warp scores
+  const int nstages = (wrows + RPS - 1) / RPS;
   auto swz_off = [&](int r, int part) { return r * RB + ((part ^ (CPR > 1 ? ((r >> 2) & (CPR - 1)) : 0)) << 4); };
-  auto issue = [&](int stage, int slot) {
-    uint8_t* dst = ring + slot * kStreamStageBytes;
-    if (seg_path) {
+  auto issue = [&](int stage) {
+    if (stage >= nstages) return;
+    uint8_t* dst = wring + (stage % kStreamStages) * kStreamStageBytes;
 #pragma unroll
-      for (int g = warp; g < kStreamStageBytes / 512; g += kIndexThreads / 32) {
-        const int r = g * (512 / RB) + seg_row;  // row within the stage
-        const int lr = stage * RPS + r;
-        const bool valid = lr < nrows;
-        const int vr = valid ? lr : 0;
-        const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + seg_part * 16;
-        cp_async_16(smem_u32(dst + swz_off(r, seg_part)), src, valid ? 16u : 0u);
-      }
-    } else {
-#pragma unroll
-      for (int c = tid; c < kStreamStageBytes / 16; c += kIndexThreads) {
-        const int r = c / CPR, part = c % CPR;
-        const int lr = stage * RPS + r;
-        const bool valid = lr < nrows;
-        const int vr = valid ? lr : 0;
-        const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + part * 16;
-        cp_async_16(smem_u32(dst + swz_off(r, part)), src, valid ? 16u : 0u);
-      }
+    for (int k = 0; k < kStreamStageBytes / 512; ++k) {
+      const int c = lane + 32 * k;  // 16-byte chunk of the stage
+      const int r = c / CPR, part = c % CPR;
+      const int lr = w0 + stage * RPS + r;
+      const bool valid = r < RPS && lr < w0 + wrows;
+      const int vr = valid ? lr : w0;
+      const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + part * 16;
+      cp_async_16(smem_u32(dst + swz_off(r, part)), src, valid ? 16u : 0u);
     }
   };
-  const int nstages = (nrows + RPS - 1) / RPS;
 #pragma unroll
   for (int st = 0; st < kStreamStages - 1; ++st) {
-    if (st < nstages) issue(st, st);
+    issue(st);
     cp_async_commit();
   }
   for (int st = 0; st < nstages; ++st) {
-    const int ns = st + kStreamStages - 1;
-    if (ns < nstages) issue(ns, ns % kStreamStages);
+    issue(st + kStreamStages - 1);
     cp_async_commit();
     cp_async_wait<kStreamStages - 1>();
-    __syncthreads();
-    const uint8_t* src = ring + (st % kStreamStages) * kStreamStageBytes;
-    uint32_t key[RPT];
+    __syncwarp();
+    const uint8_t* src = wring + (st % kStreamStages) * kStreamStageBytes;
+    uint32_t key[RPL];
     uint32_t mask = 0u;
 #pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int r = tid + k * kIndexThreads;
+    for (int k = 0; k < RPL; ++k) {
+      const int r = lane + 32 * k;
       uint32_t w[Geo::kWords];
 #pragma unroll
       for (int part = 0; part < CPR; ++part) {
@@ -632,8 +632,7 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
         w[4 * part + 3] = v.w;
       }
       key[k] = score_key(scale * row_dot<R, FP8>(w, u2));
-      const int lr = st * RPS + r;
-      if (r < RPS && lr < nrows && key[k] >= tau) mask |= 1u << k;
+      if (r < RPS && st * RPS + r < wrows && key[k] >= tau) mask |= 1u << k;
     }
     if (__ballot_sync(0xffffffffu, mask != 0u)) {
       const uint32_t mine = __popc(mask);
@@ -647,19 +646,20 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
       if (lane == 31) slot = atomicAdd(&s_ncand, incl);
       slot = __shfl_sync(0xffffffffu, slot, 31) + incl - mine;
 #pragma unroll
-      for (int k = 0; k < RPT; ++k) {
+      for (int k = 0; k < RPL; ++k) {
         if ((mask >> k) & 1u) {
           if (slot < (uint32_t)kStageCap) {
             ckey[slot] = key[k];
-            cpos[slot] = (uint32_t)(t_begin + st * RPS + tid + k * kIndexThreads);
+            cpos[slot] = (uint32_t)(t_begin + w0 + st * RPS + lane + 32 * k);
           }
           ++slot;
         }
       }
     }
-    __syncthreads();  // the slot is refilled by a later stage
+    __syncwarp();  // the slot is refilled by a later stage
   }
   cp_async_wait<0>();
+  __syncthreads();
   const uint32_t nc = s_ncand;
   if (nc == 0u) return;
   if (tid == 0) s_base = atomicAdd(&p.ccount[bh], nc <= (uint32_t)kStageCap ? nc : (uint32_t)p.cap + 1u);
@@ -952,7 +952,7 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const dim3 grid((p.max_seq_len + kStreamChunk - 1) / kStreamChunk, p.Hkv, p.B);
-  const size_t ring = (size_t)kStreamStages * kStreamStageBytes;
+  const size_t ring = (size_t)(kIndexThreads / 32) * kStreamStages * kStreamStageBytes;
   auto k = lisa_index_stream_kernel<R, FP8>;
   e = set_smem(k, ring);
   if (e != cudaSuccess) return e;

@@ -37,7 +37,10 @@ struct IndexParams {
 
 struct AttnParams {
   int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
-  int splits, split_len;
+  int npairs;   // B * Hkv
+  int tpp;      // 64-position tiles per pair: ceil(M / 64)
+  int grid;     // CTAs of the stream-K launch (<= npairs * tpp)
+  int max_seg;  // partial slots per pair: ceil(grid / npairs) + 1
   float scale_log2;  // softmax scale * log2(e)
   const int32_t* seq_lens;
   const int32_t* page_table;
@@ -46,9 +49,9 @@ struct AttnParams {
   const __nv_bfloat16* v_pool;
   const int32_t* idx;
   const int32_t* count;
-  float* o_part;   // [B][Hkv][splits][G][d], unnormalised, relative to the partition max
-  float* ml_part;  // [B][Hkv][splits][G][2]: (max in log2 units, sum of 2^(x - max))
-  uint32_t* acount;  // [B][Hkv]: partitions finished (the last one merges and resets it to 0)
+  float* o_part;   // [B][Hkv][max_seg][G][d], unnormalised, relative to the partial's max
+  float* ml_part;  // [B][Hkv][max_seg][G][2]: (max in log2 units, sum of 2^(x - max))
+  uint32_t* acount;  // [B][Hkv]: partials written (the last writer merges and resets it to 0)
   uint32_t* err;
   // Output of the merge (done by the last partition CTA of each (b, KV head)).
   __nv_bfloat16* out;
