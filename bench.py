@@ -32,7 +32,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-decode attn queries/sec at 128K ctx, M=2048; achieved HBM GB/s vs peak"
-WORKLOAD = "128K paged decode: B=16, 64q/8kv heads, d=128, n=131072, r=32 FP8 projected keys, M=2048, page 64"
+WORKLOAD = ("128K paged decode: B=16, 64q/8kv heads, d=128, n=131072, r=32 FP8 projected keys, M=2048, page 64, "
+            "K|V interleaved per row")
 FALLBACK_HBM_GBS = 6650.0
 INDEX_SOURCES = ["indexed_top_sparse_b200/csrc/lisa_index.cu", "indexed_top_sparse_b200/csrc/lisa_common.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "index_select_128k_traffic.json")
@@ -219,9 +220,11 @@ def run_ours(args, world, rank, local):
     scale = prob.kproj_scale.to(dev)
     stream = torch.cuda.current_stream(dev)
 
+    k_arg, v_arg = R.kv_args(prob)
+
     def step(events=None, q=None):
         L.lisa_fused_decode(desc, prob.q if q is None else q, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale,
-                            prob.k_pool, prob.v_pool, None, None, None, None, None, out, lse, ws, events=events,
+                            k_arg, v_arg, None, None, None, None, None, out, lse, ws, events=events,
                             stream=stream)
 
     for _ in range(args.warmup):

@@ -47,7 +47,8 @@
  *   P            fp32 [Hkv][r][d]
  *   kproj_pool   [num_pages][Hkv][page_size][r]  of uint8 E4M3 codes, or of fp32
  *   kproj_scale  fp32 [Hkv]
- *   k_pool/v_pool bf16 [num_pages][page_size][Hkv][d]
+ *   k_pool/v_pool bf16 [num_pages][page_size][Hkv][d] (separate pools), or one pool
+ *                bf16 [num_pages][page_size][Hkv][2][d] with K then V per row (kv_row_stride = 2d)
  *   page_table   int32 [B][max_pages_per_seq]: position t of sequence b lives in page page_table[b][t /
  *                page_size], slot t % page_size.  A contiguous cache is a pool with an identity table.
  *   seq_lens     int32 [B], 0 <= n_b <= max_seq_len
@@ -104,6 +105,10 @@ typedef struct {
   const int32_t* seq_lens;   /* device int32 [B]                                                   */
   const int32_t* page_table; /* device int32 [B][max_pages_per_seq]                                */
   float softmax_scale;       /* attention logit scale; <= 0 selects 1/sqrt(d)                      */
+  int32_t kv_row_stride;     /* elements from one (page, slot, KV head) row of k_pool / v_pool to
+                                the next: 0 (or d) for separate K and V pools; 2 * d for one pool
+                                holding K and V of each row side by side (v_pool = k_pool + d), the
+                                faster layout: one 512-byte read per selected position at d = 128 */
 } lisa_decode_desc;
 
 /* Optional linear-attention branch (one state per (b, KV head)); S and z are updated in place. */

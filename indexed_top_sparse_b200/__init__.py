@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     KPROJ_FP8_E4M3,
     LIB_PATH,
     DecodeDesc,
+    DevicePtr,
     LinearBranch,
     LisaError,
     StageEvents,

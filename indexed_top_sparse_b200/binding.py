@@ -60,6 +60,7 @@ class DecodeDesc(ctypes.Structure):
         ("seq_lens", ctypes.c_void_p),
         ("page_table", ctypes.c_void_p),
         ("softmax_scale", ctypes.c_float),
+        ("kv_row_stride", ctypes.c_int32),
     ]
 
 
@@ -110,9 +111,15 @@ for _name, (_res, _args) in _sig.items():
 EXPORTED = tuple(_sig)
 
 
+class DevicePtr(int):
+    """A raw device address (e.g. the V half of an interleaved K|V pool), passed through as is."""
+
+
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
+    if isinstance(t, DevicePtr):
+        return ctypes.c_void_p(int(t))
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"expected a torch.Tensor, got {type(t)}")
     if not t.is_contiguous():
@@ -138,11 +145,12 @@ def lisa_status_string(status: int) -> str:
 
 
 def make_desc(*, batch, num_q_heads, num_kv_heads, head_dim, idx_dim, budget_m, page_size, max_pages_per_seq,
-              max_seq_len, num_pages, seq_lens=None, page_table=None, softmax_scale=0.0) -> DecodeDesc:
+              max_seq_len, num_pages, seq_lens=None, page_table=None, softmax_scale=0.0,
+              kv_row_stride=0) -> DecodeDesc:
     """Fill a lisa_decode_desc.  The desc refers to (does not own) seq_lens/page_table."""
     d = DecodeDesc(
         batch, num_q_heads, num_kv_heads, head_dim, idx_dim, budget_m, page_size, max_pages_per_seq, max_seq_len,
-        num_pages, None, None, float(softmax_scale),
+        num_pages, None, None, float(softmax_scale), int(kv_row_stride),
     )
     if seq_lens is not None:
         d.seq_lens = _ptr(seq_lens).value

@@ -47,6 +47,8 @@ lisa_status check_desc(const lisa_decode_desc* d) {
   if ((unsigned long long)d->num_pages * (unsigned long long)d->page_size * (unsigned long long)d->num_kv_heads >
       0xffffffffull)
     return LISA_ERR_UNSUPPORTED;
+  if (d->kv_row_stride != 0 && (d->kv_row_stride < d->head_dim || d->kv_row_stride % 8 != 0))
+    return LISA_ERR_INVALID_ARG;  // rows must not overlap and must stay 16-byte aligned
   return LISA_OK;
 }
 
@@ -166,6 +168,7 @@ AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, con
   p.max_pages = d.max_pages_per_seq;
   p.max_seq_len = d.max_seq_len;
   p.num_pages = d.num_pages;
+  p.kv_stride_bytes = (d.kv_row_stride > 0 ? d.kv_row_stride : d.head_dim) * 2;
   p.npairs = d.batch * d.num_kv_heads;
   p.tpp = L.tpp;
   p.grid = L.grid;

@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     for (int r = tid / Geo::kChunks; r < kAttnTile; r += Geo::kRowsPerPass) {
       const uint32_t row = rows[r];
       const bool valid = row != kNoRow;
-      const size_t off = (size_t)(valid ? row : 0u) * Geo::kRowBytes + (size_t)ch * 16;
+      const size_t off = (size_t)(valid ? row : 0u) * (size_t)p.kv_stride_bytes + (size_t)ch * 16;
       const uint32_t so = swz(r, ch, Geo::kRowBytes);
       cp_async_16(smem_u32(kdst + so), kbase + off, valid ? 16u : 0u);
       cp_async_16(smem_u32(vdst + so), vbase + off, valid ? 16u : 0u);

@@ -37,6 +37,7 @@ struct IndexParams {
 
 struct AttnParams {
   int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
+  int kv_stride_bytes;  // bytes between consecutive (page, slot, KV head) rows of the K/V pools
   int npairs;   // B * Hkv
   int tpp;      // 64-position tiles per pair: ceil(M / 64)
   int grid;     // CTAs of the stream-K launch (<= npairs * tpp)

@@ -46,6 +46,8 @@ CASES = {
     "g8_ps1024": lambda dev: small(dev, B=2, Hq=16, Hkv=2, M=512, seq_lens=[20000, 2500], page_size=1024,
                                    paged=True, seed=80),
     "g1": lambda dev: small(dev, B=2, Hq=3, Hkv=3, M=300, seq_lens=[4000, 301], paged=True, seed=81),
+    "separate_kv_pools": lambda dev: small(dev, B=2, Hq=16, Hkv=2, M=700, seq_lens=[9000, 2200], paged=True,
+                                           kv_interleaved=False, seed=82),
     "c2_full": lambda dev: config2(device=dev),
 }
 

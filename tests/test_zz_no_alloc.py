@@ -40,7 +40,8 @@ def test_noalloc_attention_matches_workspace_attention_on_two_calls(cuda_device)
         want_out, want_lse = R.attention(prob, idx, count, ws, desc)
         out = torch.full_like(want_out, float("nan"))
         lse = torch.full_like(want_lse, float("nan"))
-        L.lisa_sparse_decode_attn_noalloc(desc, prob.q, prob.k_pool, prob.v_pool, idx, count, out, lse)
+        k, v = R.kv_args(prob)
+        L.lisa_sparse_decode_attn_noalloc(desc, prob.q, k, v, idx, count, out, lse)
         torch.cuda.synchronize()
         pairs = [(b, h) for b in range(prob.B) for h in range(prob.Hkv)]
         check_outputs(out.float().cpu().double().numpy(), want_out.float().cpu().double().numpy(), pairs, prob.G)

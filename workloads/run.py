@@ -20,8 +20,15 @@ def desc_of(prob: DecodeProblem) -> L.DecodeDesc:
         batch=prob.B, num_q_heads=prob.Hq, num_kv_heads=prob.Hkv, head_dim=prob.d, idx_dim=prob.r,
         budget_m=prob.M, page_size=prob.page_size, max_pages_per_seq=prob.max_pages,
         max_seq_len=prob.max_seq_len, num_pages=prob.num_pages, seq_lens=prob.seq_lens,
-        page_table=prob.page_table, softmax_scale=prob.softmax_scale,
+        page_table=prob.page_table, softmax_scale=prob.softmax_scale, kv_row_stride=prob.kv_row_stride,
     )
+
+
+def kv_args(prob: DecodeProblem):
+    """(k_pool, v_pool) arguments of the library: the interleaved pool and its V half, or the two pools."""
+    if prob.kv is not None:
+        return prob.kv, L.DevicePtr(prob.kv.data_ptr() + prob.d * prob.kv.element_size())
+    return prob.k_pool, prob.v_pool
 
 
 def kproj_dtype(prob: DecodeProblem) -> int:
@@ -60,7 +67,8 @@ def attention(prob: DecodeProblem, idx: torch.Tensor, count: torch.Tensor, ws: t
     desc = desc or desc_of(prob)
     out = torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=prob.device)
     lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=prob.device)
-    L.lisa_sparse_decode_attn(desc, prob.q, prob.k_pool, prob.v_pool, idx, count, out, lse, ws)
+    k, v = kv_args(prob)
+    L.lisa_sparse_decode_attn(desc, prob.q, k, v, idx, count, out, lse, ws)
     return out, lse
 
 
@@ -80,6 +88,7 @@ def fused(prob: DecodeProblem, ws: torch.Tensor, desc=None, reuse: Optional[tupl
         lb = L.linear_branch(lin.S, lin.z, lin.k_new, lin.v_new, lin.gate)
     ridx, rcount = (None, None) if reuse is None else reuse
     scale = prob.kproj_scale.to(dev) if prob.kproj is not None else None
-    L.lisa_fused_decode(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), scale, prob.k_pool, prob.v_pool, ridx,
+    k, v = kv_args(prob)
+    L.lisa_fused_decode(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), scale, k, v, ridx,
                         rcount, idx, count, lb, out, lse, ws, events=events, stream=stream)
     return {"out": out, "lse": lse, "idx": idx, "count": count}

@@ -6,7 +6,8 @@ Layouts (all row-major):
 * P          fp32  [Hkv][r][d]          per-KV-head basis with orthonormal rows
 * kproj      u8 (FP8 E4M3 codes) or fp32, paged: [num_pages][Hkv][page_size][r]
 * kproj_scale fp32 [Hkv]                dequantisation scale per KV head (1 for fp32)
-* k_pool, v_pool bf16, paged: [num_pages][page_size][Hkv][d]
+* k_pool, v_pool bf16, paged: [num_pages][page_size][Hkv][d] -- by default views into one pool
+                 kv [num_pages][page_size][Hkv][2][d] that holds K then V of each row
 * page_table int32 [B][max_pages]       page id of each logical page, -1 where unused
 * seq_lens   int32 [B]
 
@@ -72,7 +73,13 @@ class DecodeProblem:
     softmax_scale: float = 0.0  # 0 means 1/sqrt(d)
     planted: Optional[list] = None  # planted[b][h] -> LongTensor of positions
     lin: Optional[LinearBranchInputs] = None
+    kv: Optional[torch.Tensor] = None  # interleaved K|V pool backing k_pool / v_pool, if any
     meta: dict = field(default_factory=dict)
+
+    @property
+    def kv_row_stride(self) -> int:
+        """Elements between consecutive (page, slot, KV head) rows of the K/V pools (0: separate pools)."""
+        return 2 * self.d if self.kv is not None else 0
 
     @property
     def G(self) -> int:
@@ -84,6 +91,7 @@ class DecodeProblem:
 
     def to(self, device) -> "DecodeProblem":
         mv = lambda t: None if t is None else t.to(device)
+        kv = mv(self.kv)
         return replace(
             self,
             seq_lens=mv(self.seq_lens),
@@ -92,8 +100,9 @@ class DecodeProblem:
             P=mv(self.P),
             kproj=mv(self.kproj),
             kproj_scale=mv(self.kproj_scale),
-            k_pool=mv(self.k_pool),
-            v_pool=mv(self.v_pool),
+            k_pool=kv[:, :, :, 0] if kv is not None else mv(self.k_pool),
+            v_pool=kv[:, :, :, 1] if kv is not None else mv(self.v_pool),
+            kv=kv,
             lin=None if self.lin is None else self.lin.to(device),
         )
 
@@ -209,6 +218,7 @@ def make_problem(
     linear: bool = False,
     softmax_scale: float = 0.0,
     with_kproj: bool = True,
+    kv_interleaved: bool = True,
 ) -> DecodeProblem:
     """Draw one decode problem.
 
@@ -227,8 +237,13 @@ def make_problem(
     P = _orthonormal_basis(Hkv, r, d, _gen(seed, 3), bf16_basis)
 
     g_dev = _gen(seed, 4, device)
-    k_pool = torch.randn(num_pages, page_size, Hkv, d, generator=g_dev, device=device, dtype=torch.bfloat16)
-    v_pool = torch.randn(num_pages, page_size, Hkv, d, generator=g_dev, device=device, dtype=torch.bfloat16)
+    kv = None
+    if kv_interleaved:
+        kv = torch.randn(num_pages, page_size, Hkv, 2, d, generator=g_dev, device=device, dtype=torch.bfloat16)
+        k_pool, v_pool = kv[:, :, :, 0], kv[:, :, :, 1]
+    else:
+        k_pool = torch.randn(num_pages, page_size, Hkv, d, generator=g_dev, device=device, dtype=torch.bfloat16)
+        v_pool = torch.randn(num_pages, page_size, Hkv, d, generator=g_dev, device=device, dtype=torch.bfloat16)
 
     planted = None
     if plant[0] != "none":
@@ -306,6 +321,7 @@ def make_problem(
         softmax_scale=softmax_scale,
         planted=planted,
         lin=lin,
+        kv=kv,
         meta={"seed": seed, "paged": paged, "plant": plant},
     )
     return prob.to(device)
