@@ -123,6 +123,10 @@ typedef struct {
 /* Optional events recorded on `stream` between the stages of lisa_fused_decode (any may be NULL). */
 typedef struct {
   lisa_event_t start;       /* before the index stage (score + top-M)         */
+  lisa_event_t after_sample;/* after the threshold-sampling kernel (index stage, step 1 of 3;
+                               not recorded when indices are reused)          */
+  lisa_event_t after_stream;/* after the scoring stream kernel (index stage, step 2 of 3;
+                               not recorded when indices are reused)          */
   lisa_event_t after_index; /* after the index stage, before attention        */
   lisa_event_t after_attn;  /* after the attention kernel (which also merges the partitions and
                                applies the linear branch and gate)            */

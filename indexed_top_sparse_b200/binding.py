@@ -77,6 +77,8 @@ class LinearBranch(ctypes.Structure):
 class StageEvents(ctypes.Structure):
     _fields_ = [
         ("start", ctypes.c_void_p),
+        ("after_sample", ctypes.c_void_p),
+        ("after_stream", ctypes.c_void_p),
         ("after_index", ctypes.c_void_p),
         ("after_attn", ctypes.c_void_p),
         ("end", ctypes.c_void_p),
@@ -234,7 +236,8 @@ def linear_branch(S, z, k_new, v_new, gate_logit) -> LinearBranch:
     return lb
 
 
-def stage_events(start=None, after_index=None, after_attn=None, end=None, stream=None) -> StageEvents:
+def stage_events(start=None, after_index=None, after_attn=None, end=None, stream=None, after_sample=None,
+                 after_stream=None) -> StageEvents:
     """Stage events for lisa_fused_decode from torch.cuda.Event objects.
 
     torch creates the underlying CUDA event lazily, on its first record; each event is
@@ -248,8 +251,8 @@ def stage_events(start=None, after_index=None, after_attn=None, end=None, stream
             e.record(stream if stream is not None else torch.cuda.current_stream())
         return e.cuda_event
 
-    ev = StageEvents(h(start), h(after_index), h(after_attn), h(end))
-    ev._refs = (start, after_index, after_attn, end)
+    ev = StageEvents(h(start), h(after_sample), h(after_stream), h(after_index), h(after_attn), h(end))
+    ev._refs = (start, after_sample, after_stream, after_index, after_attn, end)
     return ev
 
 

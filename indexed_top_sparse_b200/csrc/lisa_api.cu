@@ -431,7 +431,9 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
     p.kproj_scale = kproj_scale;
     p.idx = di;
     p.count = dc;
-    LISA_TRY(cuda_status(launch_index_topm(p, st)));
+    cudaEvent_t es = events ? reinterpret_cast<cudaEvent_t>(events->after_sample) : nullptr;
+    cudaEvent_t et = events ? reinterpret_cast<cudaEvent_t>(events->after_stream) : nullptr;
+    LISA_TRY(cuda_status(launch_index_topm(p, st, es, et)));
     idx = di;
     count = dc;
   } else {

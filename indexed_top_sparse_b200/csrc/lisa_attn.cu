@@ -24,6 +24,9 @@
 //    (sequence, KV head) are merged by log-sum-exp in the CTA that writes the last of them (a fenced
 //    atomic counter, no waiting), which also runs the linear branch and the gate.
 
+#include <climits>
+#include <type_traits>
+
 #include "lisa_common.cuh"
 #include "lisa_kernels.h"
 
@@ -60,52 +63,57 @@ size_t attn_smem_bytes(int d) { return d == 64 ? AttnGeom<64>::kSmem : AttnGeom<
 __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
 // Merge the nseg partials of one (b, KV head) for its G query heads; optional linear branch + gate.
-// Run by the 128 threads of the CTA that wrote the last partial; thread e owns output column e.
+// Run by the 128 threads of a CTA that holds no copies in flight; thread e owns output column e.
+// scr: 3 * nseg * G floats of shared memory (the CTA's idle pipeline stages).
 template <int D>
-__device__ void merge_pair(const AttnParams& p, int b, int h, int nseg) {
+__device__ void merge_pair(const AttnParams& p, int b, int h, int nseg, float* scr) {
   __shared__ float fk[D];
   __shared__ float fq[kMaxG][D];
   __shared__ float zn[D];
   __shared__ float den[kMaxG];
-  __shared__ float wseg[kMaxG][64];
   __shared__ float mstar[kMaxG], lstar[kMaxG];
   const int G = p.Hq / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = (size_t)b * p.Hkv + h;
-  const float* mlp = p.ml_part + bh * p.max_seg * G * 2;
+  const float2* mlp = reinterpret_cast<const float2*>(p.ml_part) + bh * p.max_seg * G;
   const float* op = p.o_part + bh * p.max_seg * G * D;
+  float* mseg = scr;                // [nseg][G] running max of each partial
+  float* lseg = scr + nseg * G;     // [nseg][G] its sum
+  float* wseg = lseg + nseg * G;    // [nseg][G] its weight 2^(m_s - m*)
 
-  float acc[kMaxG];
-#pragma unroll
-  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  // every (max, sum) pair in flight at once
+#pragma unroll 4
+  for (int e = tid; e < nseg * G; e += blockDim.x) {
+    const float2 v = __ldcg(mlp + e);
+    mseg[e] = v.x;
+    lseg[e] = v.y;
+  }
+  __syncthreads();
   if (tid < G) {
     float mx = kNegInf;
-    for (int s = 0; s < nseg; ++s) mx = fmaxf(mx, __ldcg(&mlp[(s * G + tid) * 2]));
+    for (int s = 0; s < nseg; ++s) mx = fmaxf(mx, mseg[s * G + tid]);
     float l = 0.f;
-    if (mx != kNegInf)
-      for (int s = 0; s < nseg; ++s) {
-        const float ms = __ldcg(&mlp[(s * G + tid) * 2]);
-        if (ms != kNegInf) l += __ldcg(&mlp[(s * G + tid) * 2 + 1]) * exp2f(ms - mx);
-      }
+    for (int s = 0; s < nseg; ++s) {
+      const float ms = mseg[s * G + tid];
+      const float w = (ms != kNegInf && mx != kNegInf) ? exp2f(ms - mx) : 0.f;
+      wseg[s * G + tid] = w;
+      l += w * lseg[s * G + tid];
+    }
     mstar[tid] = mx;
     lstar[tid] = l;
   }
-  for (int s0 = 0; s0 < nseg; s0 += 64) {
-    __syncthreads();
-    for (int e = tid; e < G * 64; e += blockDim.x) {
-      const int g = e / 64, s = s0 + (e - g * 64);
-      float w = 0.f;
-      if (s < nseg) {
-        const float ms = __ldcg(&mlp[(s * G + g) * 2]);
-        if (ms != kNegInf && mstar[g] != kNegInf) w = exp2f(ms - mstar[g]);
-      }
-      wseg[g][e - g * 64] = w;
-    }
-    __syncthreads();
-    if (tid < D) {
-      const int s1 = min(nseg, s0 + 64);
-      for (int s = s0; s < s1; ++s)
-        for (int g = 0; g < G; ++g) acc[g] += wseg[g][s - s0] * __ldcg(&op[((size_t)s * G + g) * D + tid]);
+  __syncthreads();
+  float acc[kMaxG];
+#pragma unroll
+  for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
+  if (tid < D) {
+#pragma unroll 2
+    for (int s = 0; s < nseg; ++s) {
+      float v[kMaxG];
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) v[g] = g < G ? __ldcg(&op[((size_t)s * G + g) * D + tid]) : 0.f;
+#pragma unroll
+      for (int g = 0; g < kMaxG; ++g) acc[g] = fmaf(wseg[s * G + (g < G ? g : 0)], v[g], acc[g]);
     }
   }
   float sparse[kMaxG];
@@ -166,28 +174,14 @@ __device__ void merge_pair(const AttnParams& p, int b, int h, int nseg) {
   }
 }
 
-// Valid positions of (b, h): count clamped to [0, min(M, n_b)] (flagging out-of-range values).
-__device__ __forceinline__ int pair_count(const AttnParams& p, int pr, int b, bool flag) {
-  int n = p.seq_lens[b];
-  if (n < 0 || n > p.max_seq_len) {
-    if (flag) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
-    n = n < 0 ? 0 : p.max_seq_len;
-  }
-  const int limit = min(p.M, n);
-  int cnt = p.count[pr];
-  if (cnt < 0 || cnt > limit) {
-    if (flag) flag_error(p.err, LISA_DEVERR_COUNT);
-    cnt = cnt < 0 ? 0 : limit;
-  }
-  return cnt;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnParams p) {
   using Geo = AttnGeom<D>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint32_t* rows_sm = reinterpret_cast<uint32_t*>(smem + kAttnStages * Geo::kStageBytes);  // [tile][64]
-  __shared__ uint32_t s_last;
+  __shared__ uint32_t s_last;            // bit j: this CTA completes pair pr_first + j
+  __shared__ int s_cnt[kAttnMaxTiles];   // valid positions of each touched pair
+  __shared__ int s_len[kAttnMaxTiles];   // checked length of that pair's sequence
 
   const int G = p.Hq / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -200,61 +194,87 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   const uint8_t* vbase = reinterpret_cast<const uint8_t*>(p.v_pool);
   constexpr uint32_t kNoRow = 0xffffffffu;
 
-  // Pool rows (row = (page * ps + slot) * Hkv + h) of every position of this CTA's tiles, or kNoRow
-  // past the pair's count: all index loads are issued first, then all page-table loads.
-  {
-    constexpr int kPer = kAttnMaxTiles * kAttnTile / kAttnThreads;
-    int tpos[kPer];
-    uint32_t meta[kPer];  // pair-local validity and (b, h) of each slot
+  // Pairs this CTA touches: pr_first .. pr_first + npr - 1 (at most kAttnMaxTiles).
+  const int pr_first = ntile > 0 ? t_lo / p.tpp : 0;
+  const int npr = ntile > 0 ? (t_hi - 1) / p.tpp - pr_first + 1 : 0;
+  constexpr int kPer = kAttnMaxTiles * kAttnTile / kAttnThreads;  // position slots per thread
+  // Slot k of thread tid is position e = tid + k * kAttnThreads of the run (tile e / kAttnTile); the
+  // tiles of the pipeline prologue all sit in slot 0.
+  static_assert((kAttnStages - 1) * kAttnTile <= kAttnThreads, "prologue tiles must fit in slot 0");
+
+  // Round 1: the count and sequence length of each touched pair, and the index of every slot (address
+  // clamped into the pair's M entries, validity applied later), all in flight together.
+  if (tid == 0) s_last = 0u;
+  uint32_t bad = 0u;  // LISA_DEVERR_* bits seen by this thread, flagged once at the end of the prologue
+  if (tid < npr) {
+    const int pr = pr_first + tid, b = pr / p.Hkv;
+    int n = p.seq_lens[b];
+    int cnt = p.count[pr];
+    if (n < 0 || n > p.max_seq_len) {
+      bad |= LISA_DEVERR_SEQ_LEN;
+      n = n < 0 ? 0 : p.max_seq_len;
+    }
+    const int limit = min(p.M, n);
+    if (cnt < 0 || cnt > limit) {
+      bad |= LISA_DEVERR_COUNT;
+      cnt = cnt < 0 ? 0 : limit;
+    }
+    s_cnt[tid] = cnt;
+    s_len[tid] = n;
+  }
+  int tpos[kPer];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
+  for (int k = 0; k < kPer; ++k) {
+    const int e = tid + k * kAttnThreads, i = e / kAttnTile;
+    tpos[k] = 0;
+    if (i < ntile) {
+      const int gt = t_lo + i, pr = gt / p.tpp, pos = (gt - pr * p.tpp) * kAttnTile + (e % kAttnTile);
+      tpos[k] = __ldg(&p.idx[(size_t)pr * p.M + min(pos, p.M - 1)]);
+    }
+  }
+  __syncthreads();
+
+  // Round 2: page-table loads of slots [k0, k1), then their pool rows (row = (page * ps + slot) *
+  // Hkv + h, or kNoRow past the pair's count) into rows_sm.
+  auto resolve = [&](auto k0c, auto k1c) {
+    constexpr int k0 = decltype(k0c)::value, k1 = decltype(k1c)::value;
+    int pg[k1 - k0];
+#pragma unroll
+    for (int k = k0; k < k1; ++k) {
       const int e = tid + k * kAttnThreads, i = e / kAttnTile;
-      tpos[k] = -1;
-      meta[k] = 0u;
+      pg[k - k0] = -1;
       if (i < ntile) {
-        const int gt = t_lo + i, pr = gt / p.tpp, lt = gt - pr * p.tpp;
-        const int b = pr / p.Hkv;
-        const int cnt = pair_count(p, pr, b, (e % kAttnTile) == 0 && lt == 0);
-        const int pos = lt * kAttnTile + (e % kAttnTile);
-        if (pos < cnt) {
-          tpos[k] = p.idx[(size_t)pr * p.M + pos];
-          meta[k] = 1u;
+        const int gt = t_lo + i, pr = gt / p.tpp, j = pr - pr_first;
+        const int pos = (gt - pr * p.tpp) * kAttnTile + (e % kAttnTile);
+        if (pos < s_cnt[j]) {
+          if (tpos[k] < 0 || tpos[k] >= s_len[j]) {
+            bad |= LISA_DEVERR_INDEX;
+            tpos[k] = 0;
+          }
+          const int b = pr / p.Hkv;
+          pg[k - k0] = p.page_table[(size_t)b * p.max_pages + (tpos[k] >> p.log2ps)];
+          if (pg[k - k0] < 0) pg[k - k0] = INT_MAX;  // flagged below; -1 marks "no row"
         }
       }
     }
-    int pgs[kPer];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int e = tid + k * kAttnThreads, i = e / kAttnTile;
-      pgs[k] = 0;
-      if (meta[k]) {
-        const int gt = t_lo + i, pr = gt / p.tpp, b = pr / p.Hkv;
-        const int n = min(max(p.seq_lens[b], 0), p.max_seq_len);
-        if (tpos[k] < 0 || tpos[k] >= n) {
-          flag_error(p.err, LISA_DEVERR_INDEX);
-          tpos[k] = 0;
-        }
-        pgs[k] = p.page_table[(size_t)b * p.max_pages + (tpos[k] >> p.log2ps)];
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
+    for (int k = k0; k < k1; ++k) {
       const int e = tid + k * kAttnThreads, i = e / kAttnTile;
       if (i < ntile) {
         uint32_t row = kNoRow;
-        if (meta[k]) {
-          const int gt = t_lo + i, pr = gt / p.tpp, h = pr % p.Hkv;
-          int pg = pgs[k];
-          if (pg < 0 || pg >= p.num_pages) {
-            flag_error(p.err, LISA_DEVERR_PAGE_ID);
-            pg = 0;
+        int pgk = pg[k - k0];
+        if (pgk >= 0) {
+          if (pgk >= p.num_pages) {
+            bad |= LISA_DEVERR_PAGE_ID;
+            pgk = 0;
           }
-          row = ((uint32_t)pg * (uint32_t)p.ps + (uint32_t)(tpos[k] & (p.ps - 1))) * (uint32_t)p.Hkv + (uint32_t)h;
+          const int gt = t_lo + i, pr = gt / p.tpp, h = pr % p.Hkv;
+          row = ((uint32_t)pgk * (uint32_t)p.ps + (uint32_t)(tpos[k] & (p.ps - 1))) * (uint32_t)p.Hkv + (uint32_t)h;
         }
         rows_sm[e] = row;
       }
     }
-  }
+  };
   // 16-byte cp.async copies of tile i's K and V rows into stage i % kAttnStages (zeros past the count).
   auto issue = [&](int i) {
     if (i >= ntile) return;
@@ -266,29 +286,36 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     for (int r = tid / Geo::kChunks; r < kAttnTile; r += Geo::kRowsPerPass) {
       const uint32_t row = rows[r];
       const bool valid = row != kNoRow;
-      const size_t off = (size_t)(valid ? row : 0u) * (size_t)p.kv_stride_bytes + (size_t)ch * 16;
+      const size_t off = (size_t)(valid ? row : 0u) * (uint32_t)p.kv_stride_bytes + (uint32_t)(ch * 16);
       const uint32_t so = swz(r, ch, Geo::kRowBytes);
       cp_async_16(smem_u32(kdst + so), kbase + off, valid ? 16u : 0u);
       cp_async_16(smem_u32(vdst + so), vbase + off, valid ? 16u : 0u);
     }
   };
 
+  resolve(std::integral_constant<int, 0>{}, std::integral_constant<int, 1>{});
   __syncthreads();
 #pragma unroll
   for (int st = 0; st < kAttnStages - 1; ++st) {
     issue(st);
     cp_async_commit();
   }
+  // The remaining rows resolve while the prologue tiles are in flight.
+  resolve(std::integral_constant<int, 1>{}, std::integral_constant<int, kPer>{});
+  if (bad & LISA_DEVERR_SEQ_LEN) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
+  if (bad & LISA_DEVERR_COUNT) flag_error(p.err, LISA_DEVERR_COUNT);
+  if (bad & LISA_DEVERR_INDEX) flag_error(p.err, LISA_DEVERR_INDEX);
+  if (bad & LISA_DEVERR_PAGE_ID) flag_error(p.err, LISA_DEVERR_PAGE_ID);
+  __syncthreads();
 
   float m_run[2], l_run[2];  // per head 2t_, 2t_+1 (log2 units); l is a partial over this lane's rows
   float o[D / 16][4];
   uint32_t qf[D / 16][2];  // Q^T fragments (B operand, k = d, n = query head of the group)
   int cur = -1, cur_cnt = 0;
 
-  // Write the CTA's partial for pair pr (its warps merged in shared memory at `scratch`) and, if it
-  // is the last of the pair's partials, merge them into the output.
+  // Write the CTA's partial (max, sum, unnormalised output) for pair pr, its four warps combined in
+  // shared memory at `scratch`.  Publication and merging wait for the end of the CTA's run.
   auto flush = [&](int pr, uint8_t* scratch) {
-    const int b = pr / p.Hkv, h = pr - b * p.Hkv;
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
@@ -312,9 +339,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
       wl[warp * kMaxG + 2 * t_ + 1] = l_run[1];
     }
     __syncthreads();
-    const long long first = (long long)pr * p.tpp;
-    const int c_first = owner_cta(first, T, C);
-    const int nseg = owner_cta(first + p.tpp - 1, T, C) - c_first + 1;
+    const int c_first = owner_cta((long long)pr * p.tpp, T, C);
     const size_t part = (size_t)pr * p.max_seg + (c - c_first);
     float* op = p.o_part + part * G * D;
     for (int e = tid; e < G * D; e += kAttnThreads) {
@@ -342,19 +367,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
           if (mw != kNegInf) l += wl[w * kMaxG + tid] * exp2f(mw - mx);
         }
       }
-      p.ml_part[(part * G + tid) * 2 + 0] = mx;
-      p.ml_part[(part * G + tid) * 2 + 1] = l;
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      s_last = atomicAdd(&p.acount[pr], 1u) == (uint32_t)nseg - 1u;
-      if (s_last) p.acount[pr] = 0u;
-    }
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      merge_pair<D>(p, b, h, nseg);
+      reinterpret_cast<float2*>(p.ml_part)[part * G + tid] = make_float2(mx, l);
     }
     __syncthreads();  // the scratch stage is refilled next
   };
@@ -366,7 +379,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
       if (cur >= 0) flush(cur, smem + ((i + kAttnStages - 1) % kAttnStages) * Geo::kStageBytes);
       cur = pr;
       const int b = pr / p.Hkv, h = pr - b * p.Hkv;
-      cur_cnt = pair_count(p, pr, b, false);
+      cur_cnt = s_cnt[pr - pr_first];
       const __nv_bfloat16* qrow = p.q + ((size_t)b * p.Hq + (size_t)h * G + (g_ < G ? g_ : 0)) * D;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -440,7 +453,32 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     __syncthreads();  // the stage is refilled by a later iteration
   }
   cp_async_wait<0>();
-  if (cur >= 0) flush(cur, smem + ((ntile - 1) % kAttnStages) * Geo::kStageBytes);
+  if (cur >= 0) flush(cur, smem);
+  // One release per pair this CTA touched (partials written above, ordered by the barrier that ends
+  // flush); the CTA whose arrival completes a pair's count merges that pair.
+  if (tid < npr) {
+    const int pr = pr_first + tid;
+    const long long first = (long long)pr * p.tpp;
+    const int nseg = owner_cta(first + p.tpp - 1, T, C) - owner_cta(first, T, C) + 1;
+    __threadfence();
+    if (atomicAdd(&p.acount[pr], 1u) == (uint32_t)nseg - 1u) {
+      p.acount[pr] = 0u;  // ready for the next launch
+      atomicOr(&s_last, 1u << tid);
+    }
+  }
+  __syncthreads();
+  const uint32_t mine = s_last;
+  if (mine != 0u) {
+    __threadfence();
+    for (int j = 0; j < npr; ++j) {
+      if (!((mine >> j) & 1u)) continue;
+      const int pr = pr_first + j, b = pr / p.Hkv, h = pr - b * p.Hkv;
+      const long long first = (long long)pr * p.tpp;
+      const int nseg = owner_cta(first + p.tpp - 1, T, C) - owner_cta(first, T, C) + 1;
+      merge_pair<D>(p, b, h, nseg, reinterpret_cast<float*>(smem));
+      __syncthreads();
+    }
+  }
 }
 
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream) {

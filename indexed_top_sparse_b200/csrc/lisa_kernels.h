@@ -70,7 +70,9 @@ size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
-cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream);
+// after_sample / after_stream: optional events recorded between the three kernels (nullptr: none).
+cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample = nullptr,
+                              cudaEvent_t after_stream = nullptr);
 size_t finish_smem_bytes(int max_seq_len, int cap);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
 

@@ -214,6 +214,20 @@ def test_fused_is_deterministic(cuda_device):
     assert torch.equal(a["idx"], b["idx"]) and torch.equal(a["out"], b["out"]) and torch.equal(a["lse"], b["lse"])
 
 
+
+def test_stage_events_are_recorded_in_order(cuda_device):
+    prob = small(cuda_device, seed=95)
+    ws = R.workspace(prob)
+    plain = R.fused(prob, ws)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    se = L.stage_events(start=ev[0], after_sample=ev[1], after_stream=ev[2], after_index=ev[3], after_attn=ev[4],
+                        end=ev[5])
+    timed = R.fused(prob, ws, events=se)
+    torch.cuda.synchronize()
+    gaps = [ev[i].elapsed_time(ev[i + 1]) for i in range(5)]
+    assert all(g >= 0 for g in gaps) and ev[0].elapsed_time(ev[5]) > 0
+    assert torch.equal(plain["idx"], timed["idx"]) and torch.equal(plain["out"], timed["out"])
+
 def test_empty_sequence(cuda_device):
     prob = small(cuda_device, seq_lens=[3000, 1], seed=93)
     prob.seq_lens[1] = 0
