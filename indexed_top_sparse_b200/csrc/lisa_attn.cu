@@ -62,9 +62,17 @@ size_t attn_smem_bytes(int d) { return d == 64 ? AttnGeom<64>::kSmem : AttnGeom<
 
 __device__ __forceinline__ float phi_elu1(float x) { return x > 0.f ? x + 1.f : expf(x); }
 
+constexpr int kMergeChunk = 8;  // partial outputs staged in shared memory at a time
+
+// Shared memory merge_pair needs for up to kMaxBudget / kAttnTile partials (fits the idle stages).
+template <int D>
+__host__ __device__ constexpr size_t merge_scratch_bytes() {
+  return (size_t)(3 * (kMaxBudget / kAttnTile) * kMaxG + kMergeChunk * kMaxG * D) * sizeof(float);
+}
+
 // Merge the nseg partials of one (b, KV head) for its G query heads; optional linear branch + gate.
 // Run by the 128 threads of a CTA that holds no copies in flight; thread e owns output column e.
-// scr: 3 * nseg * G floats of shared memory (the CTA's idle pipeline stages).
+// scr: merge_scratch_bytes<D>() of shared memory (the CTA's idle pipeline stages).
 template <int D>
 __device__ void merge_pair(const AttnParams& p, int b, int h, int nseg, float* scr) {
   __shared__ float fk[D];
@@ -80,8 +88,17 @@ __device__ void merge_pair(const AttnParams& p, int b, int h, int nseg, float* s
   float* mseg = scr;                // [nseg][G] running max of each partial
   float* lseg = scr + nseg * G;     // [nseg][G] its sum
   float* wseg = lseg + nseg * G;    // [nseg][G] its weight 2^(m_s - m*)
+  float* ochunk = scr + 3 * (kMaxBudget / kAttnTile) * kMaxG;  // [kMergeChunk][G][D] partial outputs
+  // Partial outputs of segments [s0, s0 + kMergeChunk) -> ochunk (16-byte cp.async through L2).
+  auto stage_outputs = [&](int s0) {
+    const int ns = min(kMergeChunk, nseg - s0);
+    const float* src = op + (size_t)s0 * G * D;
+    for (int e = tid; e < ns * G * D / 4; e += blockDim.x) cp_async_16(smem_u32(ochunk + 4 * e), src + 4 * e, 16u);
+    cp_async_commit();
+  };
 
-  // every (max, sum) pair in flight at once
+  // The first partial outputs and every (max, sum) pair in flight at once.
+  stage_outputs(0);
 #pragma unroll 4
   for (int e = tid; e < nseg * G; e += blockDim.x) {
     const float2 v = __ldcg(mlp + e);
@@ -106,14 +123,20 @@ __device__ void merge_pair(const AttnParams& p, int b, int h, int nseg, float* s
   float acc[kMaxG];
 #pragma unroll
   for (int g = 0; g < kMaxG; ++g) acc[g] = 0.f;
-  if (tid < D) {
-#pragma unroll 2
-    for (int s = 0; s < nseg; ++s) {
-      float v[kMaxG];
+  for (int s0 = 0; s0 < nseg; s0 += kMergeChunk) {
+    if (s0 > 0) {
+      __syncthreads();  // the previous chunk is consumed
+      stage_outputs(s0);
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (tid < D) {
+      const int s1 = min(nseg, s0 + kMergeChunk);
+      for (int s = s0; s < s1; ++s) {
 #pragma unroll
-      for (int g = 0; g < kMaxG; ++g) v[g] = g < G ? __ldcg(&op[((size_t)s * G + g) * D + tid]) : 0.f;
-#pragma unroll
-      for (int g = 0; g < kMaxG; ++g) acc[g] = fmaf(wseg[s * G + (g < G ? g : 0)], v[g], acc[g]);
+        for (int g = 0; g < kMaxG; ++g)
+          if (g < G) acc[g] = fmaf(wseg[s * G + g], ochunk[((s - s0) * G + g) * D + tid], acc[g]);
+      }
     }
   }
   float sparse[kMaxG];
@@ -193,6 +216,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   const uint8_t* kbase = reinterpret_cast<const uint8_t*>(p.k_pool);
   const uint8_t* vbase = reinterpret_cast<const uint8_t*>(p.v_pool);
   constexpr uint32_t kNoRow = 0xffffffffu;
+
+  static_assert(merge_scratch_bytes<D>() <= (size_t)kAttnStages * Geo::kStageBytes, "merge scratch");
+  pdl_wait();  // indices and counts come from the previous kernel
+  pdl_trigger();
 
   // Pairs this CTA touches: pr_first .. pr_first + npr - 1 (at most kAttnMaxTiles).
   const int pr_first = ntile > 0 ? t_lo / p.tpp : 0;
@@ -486,14 +513,13 @@ cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream) {
     auto k = lisa_sparse_attn_kernel<64>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<64>::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<p.grid, kAttnThreads, AttnGeom<64>::kSmem, stream>>>(p);
+    return launch_pdl(k, dim3(p.grid), dim3(kAttnThreads), AttnGeom<64>::kSmem, stream, p);
   } else {
     auto k = lisa_sparse_attn_kernel<128>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AttnGeom<128>::kSmem);
     if (e != cudaSuccess) return e;
-    k<<<p.grid, kAttnThreads, AttnGeom<128>::kSmem, stream>>>(p);
+    return launch_pdl(k, dim3(p.grid), dim3(kAttnThreads), AttnGeom<128>::kSmem, stream, p);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace lisa

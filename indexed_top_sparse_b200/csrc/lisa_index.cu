@@ -98,6 +98,91 @@ __device__ __forceinline__ float row_dot(const uint32_t* w, const float2* u2) {
   return (a0.x + a1.x) + (a0.y + a1.y);
 }
 
+// Four E4M3 values packed in a word -> two f16x2 words (bytes 0,1 -> lo; bytes 2,3 -> hi); exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 b0, b1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, b0;\n\tcvt.rn.f16x2.e4m3x2 %1, b1;\n\t}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// D(16x8 fp32) += A(16x16 f16, row) * B(16x8 f16, col).
+__device__ __forceinline__ void mma_f16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Projected-key scores of FP8 rows on the tensor cores.  The score is a dot product over the r
+// index dimensions, so the order of those dimensions is free: lane (g, t) of a warp (g = lane / 4,
+// t = lane % 4) takes the r/4 contiguous bytes [t r/4, (t+1) r/4) of rows g and g + 8 of a 16-row
+// tile as its A fragments (E4M3 -> f16 is exact), and the B fragments hold u, in the same order, as
+// two f16 parts u = 2^E (u_hi + u_lo): column pairs (2j, 2j+1) carry (u_hi, u_lo), so every lane
+// finds <c, u_hi> + <c, u_lo> of its two rows in D.  Products of f16 values are exact in the fp32
+// accumulators, and u_hi + u_lo carries u to about 2^-22, so the scores agree with an fp32 dot
+// product to fp32 rounding.  2^E keeps max |u| 2^-E in [2^13, 2^14), well inside the f16 range.
+template <int R>
+struct MmaScore {
+  static constexpr int kSteps = R / 16;  // k-steps of 16 dimensions per 16-row tile
+  uint32_t b[kSteps][2];                  // B fragments
+  float fac;                              // kproj_scale[h] * 2^E
+
+  __device__ __forceinline__ void init(const float* u, float scale, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float mx = 0.f;
+#pragma unroll
+    for (int i = 0; i < R; ++i) mx = fmaxf(mx, fabsf(u[i]));
+    const int E = mx > 0.f ? ilogbf(mx) - 13 : 0;
+    fac = scale * ldexpf(1.f, E);
+#pragma unroll
+    for (int ks = 0; ks < kSteps; ++ks) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int e0 = (R / 4) * t + 4 * ks + 2 * j;  // physical dimensions e0, e0 + 1
+        __half v[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float x = ldexpf(u[e0 + q], -E);
+          const __half hi = __float2half_rn(x);
+          v[q] = (g & 1) ? __float2half_rn(x - __half2float(hi)) : hi;
+        }
+        b[ks][j] = (uint32_t)__half_as_ushort(v[0]) | ((uint32_t)__half_as_ushort(v[1]) << 16);
+      }
+    }
+  }
+
+  // D of one 16-row tile whose row i starts at rows + i * R (shared memory, R bytes per row).
+  __device__ __forceinline__ void tile(const uint8_t* rows, int lane, float* d) const {
+    const int g = lane >> 2, t = lane & 3;
+    d[0] = d[1] = d[2] = d[3] = 0.f;
+    const uint8_t* r0 = rows + g * R + (R / 4) * t;
+    const uint8_t* r1 = r0 + 8 * R;
+    if constexpr (R == 32) {
+      const uint2 x0 = *reinterpret_cast<const uint2*>(r0);
+      const uint2 x1 = *reinterpret_cast<const uint2*>(r1);
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_f16x2(x0.x, a0, a2);
+      e4m3x4_to_f16x2(x1.x, a1, a3);
+      mma_f16_16816(d, a0, a1, a2, a3, b[0][0], b[0][1]);
+      e4m3x4_to_f16x2(x0.y, a0, a2);
+      e4m3x4_to_f16x2(x1.y, a1, a3);
+      mma_f16_16816(d, a0, a1, a2, a3, b[1][0], b[1][1]);
+    } else {
+      static_assert(R == 16, "FP8 projected keys have r = 16 or 32");
+      const uint32_t x0 = *reinterpret_cast<const uint32_t*>(r0);
+      const uint32_t x1 = *reinterpret_cast<const uint32_t*>(r1);
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_f16x2(x0, a0, a2);
+      e4m3x4_to_f16x2(x1, a1, a3);
+      mma_f16_16816(d, a0, a1, a2, a3, b[0][0], b[0][1]);
+    }
+  }
+};
+
 __device__ __forceinline__ int load_seq_len(const IndexParams& p, int b) {
   int n = p.seq_lens[b];
   if (n < 0 || n > p.max_seq_len) {
@@ -322,6 +407,15 @@ __device__ __forceinline__ void load_u2(const float* u, float2* u2) {
 }
 
 constexpr int kSampleThreads = 512;
+constexpr int kSampleRun = 8;  // adjacent positions per sampled run (one 256-byte read at r = 32 FP8)
+
+// Position of sample j of S (S = min(n, kSampleMax)): every position when n <= kSampleMax, else runs
+// of kSampleRun adjacent positions, one run starting every n / (S / kSampleRun) positions.  Runs keep
+// the DRAM reads few and whole-sector; the threshold only needs a rough quantile.
+__device__ __forceinline__ int sample_pos(int j, int n, int S) {
+  if (n <= kSampleMax) return j;
+  return (int)(((long long)(j / kSampleRun) * n) / (S / kSampleRun)) + (j % kSampleRun);
+}
 
 template <int R, bool FP8>
 __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(IndexParams p) {
@@ -332,19 +426,93 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   __shared__ uint32_t scan[32];
   __shared__ uint32_t digit[2];
   using Geo = RowGeom<R, FP8>;
-  constexpr int kSampleUnroll = Geo::kWords >= 32 ? 1 : 32 / Geo::kWords;  // rows in flight per thread
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  constexpr int SPT = kSampleMax / kSampleThreads;  // samples per thread
+  constexpr int kPW = 32 / (kSampleThreads / 32);   // rows of P per warp (r <= 32)
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * p.Hkv + h;
+  pdl_wait();  // first kernel of the step: everything it reads may come from earlier stream work
+  pdl_trigger();
   const int n = load_seq_len(p, b);
+  const int G = p.Hq / p.Hkv;
+  const int S = min(n, kSampleMax);
+  const bool sampling = n > p.M;
+  uint32_t bad = 0u;
+
+  // Round 1, all independent: the G query rows of the group (thread i < d sums column i), this
+  // warp's rows of P, and the page ids of this thread's sampled positions t_j = j n / S.
+  float qsum = 0.f;
+  if (tid < p.d) {
+    const __nv_bfloat16* qg = p.q + ((size_t)b * p.Hq + (size_t)h * G) * p.d + tid;
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) qsum += __bfloat162float(qg[(size_t)g * p.d]);
+  }
+  float prow[kPW][4];  // P[h][warp + 16 w][lane + 32 i]
+#pragma unroll
+  for (int w = 0; w < kPW; ++w) {
+    const int j = warp + (kSampleThreads / 32) * w;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      prow[w][i] = (j < p.r && c < p.d) ? __ldg(&p.P[((size_t)h * p.r + j) * p.d + c]) : 0.f;
+    }
+  }
+  int pg[SPT];
+#pragma unroll
+  for (int k = 0; k < SPT; ++k) {
+    const int j = tid + k * kSampleThreads;
+    pg[k] = 0;
+    if (sampling && j < S) {
+      const int t = sample_pos(j, n, S);
+      pg[k] = p.page_table[(size_t)b * p.max_pages + (t >> p.log2ps)];
+    }
+  }
   for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
-  compute_projected_query(p, b, h, qbar, u);  // ends with a barrier
+  if (tid < p.d) qbar[tid] = qsum / (float)G;
+
+  // Round 2: the sampled rows, KB at a time (all of them for FP8 rows), the first batch in flight
+  // while u = P qbar is formed.
+  constexpr int KB = (64 / Geo::kWords) < SPT ? (64 / Geo::kWords) : SPT;
+  uint32_t w[KB][Geo::kWords];
+  auto load_batch = [&](int k0) {
+#pragma unroll
+    for (int k = 0; k < KB; ++k) {
+      const int j = tid + (k0 + k) * kSampleThreads;
+      if (sampling && j < S) {
+        const int t = sample_pos(j, n, S);
+        int pgk = pg[k0 + k];
+        if (pgk < 0 || pgk >= p.num_pages) {
+          bad |= LISA_DEVERR_PAGE_ID;
+          pgk = 0;
+        }
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.kproj) +
+                             ((((size_t)pgk * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1))) * Geo::kRowBytes;
+#pragma unroll
+        for (int l = 0; l < Geo::kLoads; ++l) load_vec<Geo::kVec>(src + l * Geo::kVec, &w[k][l * (Geo::kVec / 4)]);
+      }
+    }
+  };
+  load_batch(0);
+  __syncthreads();
+#pragma unroll
+  for (int wr = 0; wr < kPW; ++wr) {
+    const int j = warp + (kSampleThreads / 32) * wr;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      if (c < p.d) acc = fmaf(prow[wr][i], qbar[c], acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0 && j < p.r) u[j] = acc;
+  }
+  __syncthreads();
   if (tid < p.r) p.uq[bh * 32 + tid] = u[tid];
   if (tid == 0) {
     p.ccount[bh] = 0u;
     p.done[bh] = 0u;
     p.acount[bh] = 0u;
   }
-  if (n <= p.M) {  // every position is kept; the streaming kernel skips this pair
+  if (!sampling) {  // every position is kept; the streaming kernel skips this pair
     int32_t* idx_out = p.idx + bh * p.M;
     for (int i = tid; i < p.M; i += blockDim.x) idx_out[i] = i < n ? i : -1;
     if (tid == 0) {
@@ -356,17 +524,12 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   float2 u2[R / 2];
   load_u2<R>(u, u2);
   const float scale = p.kproj_scale[h];
-  const int S = min(n, kSampleMax);
-  for (int j0 = tid; j0 < S; j0 += kSampleThreads * kSampleUnroll) {
-    uint32_t w[kSampleUnroll][Geo::kWords];
+#pragma unroll 1
+  for (int k0 = 0; k0 < SPT; k0 += KB) {
+    if (k0 > 0) load_batch(k0);
 #pragma unroll
-    for (int k = 0; k < kSampleUnroll; ++k) {
-      const int j = j0 + k * kSampleThreads;
-      if (j < S) load_row<R, FP8>(p, b, h, (int)(((long long)j * n) / S), w[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < kSampleUnroll; ++k) {
-      const int j = j0 + k * kSampleThreads;
+    for (int k = 0; k < KB; ++k) {
+      const int j = tid + (k0 + k) * kSampleThreads;
       if (j < S) {
         const uint32_t key = score_key(scale * row_dot<R, FP8>(w[k], u2));
         skey[j] = key;
@@ -374,6 +537,7 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
       }
     }
   }
+  if (bad) flag_error(p.err, bad);
   __syncthreads();
   // tau: lower edge of the 22-bit key bin that holds the rank-th largest sample key
   const uint32_t rank = (uint32_t)min((long long)S, (2LL * p.M * S + n - 1) / n + 16);
@@ -581,17 +745,17 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
       pbase[i] = base + ((((size_t)pid * p.Hkv + h) << p.log2ps) * RB);
     }
   }
-  const uint32_t tau = p.tau[bh];
-  const float scale = p.kproj_scale[h];
-  float2 u2[R / 2];
-  load_u2<R>(p.uq + bh * 32, u2);
   __syncthreads();
 
   uint8_t* wring = ring + warp * (kStreamStages * kStreamStageBytes);
   const int w0 = warp * WROWS;                               // first row of this warp (chunk-relative)
   const int wrows = max(0, min(nrows - w0, WROWS));          // rows this warp scores
   const int nstages = (wrows + RPS - 1) / RPS;
-  auto swz_off = [&](int r, int part) { return r * RB + ((part ^ (CPR > 1 ? ((r >> 2) & (CPR - 1)) : 0)) << 4); };
+  // FP8 rows are read as 16-row tensor-core tiles (8 consecutive rows per lane group: no bank
+  // conflicts unswizzled); fp32 rows are read one per lane, with 16-byte chunks XOR-swizzled.
+  auto swz_off = [&](int r, int part) {
+    return r * RB + ((part ^ (!FP8 && CPR > 1 ? ((r >> 2) & (CPR - 1)) : 0)) << 4);
+  };
   auto issue = [&](int stage) {
     if (stage >= nstages) return;
     uint8_t* dst = wring + (stage % kStreamStages) * kStreamStageBytes;
@@ -611,28 +775,70 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
     issue(st);
     cp_async_commit();
   }
+  // The projected keys are inputs of the step: their first stages are in flight before the
+  // threshold and the projected query of the sample kernel are awaited.
+  pdl_wait();
+  pdl_trigger();
+  const uint32_t tau = p.tau[bh];
+  const float scale = p.kproj_scale[h];
+  constexpr int NK = FP8 ? 2 * (RPS / 64) : RPL;  // rows a lane keys per stage
+  float2 u2[FP8 ? 1 : R / 2];
+  MmaScore<R> mma_score;
+  if constexpr (FP8)
+    mma_score.init(p.uq + bh * 32, scale, lane);
+  else
+    load_u2<R>(p.uq + bh * 32, u2);
   for (int st = 0; st < nstages; ++st) {
     issue(st + kStreamStages - 1);
     cp_async_commit();
     cp_async_wait<kStreamStages - 1>();
     __syncwarp();
     const uint8_t* src = wring + (st % kStreamStages) * kStreamStageBytes;
-    uint32_t key[RPL];
+    uint32_t key[NK];
+    int rloc[NK];  // stage-local row of key[k]
     uint32_t mask = 0u;
+    if constexpr (FP8) {
+      // 16-row tiles on the tensor cores; lane (g, t) keys rows g and g + 8 of tiles t, t + 4, ...
+      constexpr int MT = RPS / 16;
+      float d[MT][4];
 #pragma unroll
-    for (int k = 0; k < RPL; ++k) {
-      const int r = lane + 32 * k;
-      uint32_t w[Geo::kWords];
+      for (int mt = 0; mt < MT; ++mt) mma_score.tile(src + mt * 16 * RB, lane, d[mt]);
+      const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-      for (int part = 0; part < CPR; ++part) {
-        const uint4 v = r < RPS ? *reinterpret_cast<const uint4*>(src + swz_off(r, part)) : make_uint4(0u, 0u, 0u, 0u);
-        w[4 * part + 0] = v.x;
-        w[4 * part + 1] = v.y;
-        w[4 * part + 2] = v.z;
-        w[4 * part + 3] = v.w;
+      for (int o = 0; o < MT / 4; ++o) {
+        float s0 = d[4 * o][0] + d[4 * o][1], s1 = d[4 * o][2] + d[4 * o][3];
+#pragma unroll
+        for (int q = 1; q < 4; ++q) {
+          if (t == q) {
+            s0 = d[4 * o + q][0] + d[4 * o + q][1];
+            s1 = d[4 * o + q][2] + d[4 * o + q][3];
+          }
+        }
+        rloc[2 * o] = (4 * o + t) * 16 + g;
+        rloc[2 * o + 1] = rloc[2 * o] + 8;
+        key[2 * o] = score_key(mma_score.fac * s0);
+        key[2 * o + 1] = score_key(mma_score.fac * s1);
       }
-      key[k] = score_key(scale * row_dot<R, FP8>(w, u2));
-      if (r < RPS && st * RPS + r < wrows && key[k] >= tau) mask |= 1u << k;
+#pragma unroll
+      for (int k = 0; k < NK; ++k)
+        if (st * RPS + rloc[k] < wrows && key[k] >= tau) mask |= 1u << k;
+    } else {
+#pragma unroll
+      for (int k = 0; k < NK; ++k) {
+        const int r = lane + 32 * k;
+        rloc[k] = r;
+        uint32_t w[Geo::kWords];
+#pragma unroll
+        for (int part = 0; part < CPR; ++part) {
+          const uint4 v = r < RPS ? *reinterpret_cast<const uint4*>(src + swz_off(r, part)) : make_uint4(0u, 0u, 0u, 0u);
+          w[4 * part + 0] = v.x;
+          w[4 * part + 1] = v.y;
+          w[4 * part + 2] = v.z;
+          w[4 * part + 3] = v.w;
+        }
+        key[k] = score_key(scale * row_dot<R, FP8>(w, u2));
+        if (r < RPS && st * RPS + r < wrows && key[k] >= tau) mask |= 1u << k;
+      }
     }
     if (__ballot_sync(0xffffffffu, mask != 0u)) {
       const uint32_t mine = __popc(mask);
@@ -646,11 +852,11 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
       if (lane == 31) slot = atomicAdd(&s_ncand, incl);
       slot = __shfl_sync(0xffffffffu, slot, 31) + incl - mine;
 #pragma unroll
-      for (int k = 0; k < RPL; ++k) {
+      for (int k = 0; k < NK; ++k) {
         if ((mask >> k) & 1u) {
           if (slot < (uint32_t)kStageCap) {
             ckey[slot] = key[k];
-            cpos[slot] = (uint32_t)(t_begin + w0 + st * RPS + lane + 32 * k);
+            cpos[slot] = (uint32_t)(t_begin + w0 + st * RPS + rloc[k]);
           }
           ++slot;
         }
@@ -922,6 +1128,8 @@ __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(Index
   const int h = blockIdx.x, b = blockIdx.y;
   const int n = load_seq_len(p, b);
   if (n <= p.M) return;  // the sample kernel wrote the full set
+  pdl_wait();  // candidates and counts come from the streaming kernel
+  pdl_trigger();
   uint32_t* cstage = fsm + 2 * finish_bitmap_words(p.max_seq_len);
   finish_pair<R, FP8, kFinishThreads>(p, b, h, n, fsm, cstage, finish_stage_cap(p.cap));
 }
@@ -947,29 +1155,31 @@ cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStre
 }
 
 template <int R, bool FP8>
-static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream) {
-  lisa_index_sample_kernel<R, FP8><<<dim3(p.Hkv, p.B), kSampleThreads, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample,
+                                 cudaEvent_t after_stream) {
+  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, FP8>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
+  if (after_sample != nullptr && (e = cudaEventRecord(after_sample, stream)) != cudaSuccess) return e;
   const dim3 grid((p.max_seq_len + kStreamChunk - 1) / kStreamChunk, p.Hkv, p.B);
   const size_t ring = (size_t)(kIndexThreads / 32) * kStreamStages * kStreamStageBytes;
   auto k = lisa_index_stream_kernel<R, FP8>;
   e = set_smem(k, ring);
   if (e != cudaSuccess) return e;
-  k<<<grid, kIndexThreads, ring, stream>>>(p);
-  e = cudaGetLastError();
+  e = launch_pdl(k, grid, dim3(kIndexThreads), ring, stream, p);
   if (e != cudaSuccess) return e;
+  if (after_stream != nullptr && (e = cudaEventRecord(after_stream, stream)) != cudaSuccess) return e;
   const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap);
   auto f = lisa_index_finish_kernel<R, FP8>;
   e = set_smem(f, fs);
   if (e != cudaSuccess) return e;
-  f<<<dim3(p.Hkv, p.B), kFinishThreads, fs, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);
 }
 
-cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream) {
-  if (p.kproj_fp8) return p.r == 16 ? launch_topm_t<16, true>(p, stream) : launch_topm_t<32, true>(p, stream);
-  return p.r == 16 ? launch_topm_t<16, false>(p, stream) : launch_topm_t<32, false>(p, stream);
+cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample,
+                              cudaEvent_t after_stream) {
+  const cudaEvent_t a = after_sample, b = after_stream;
+  if (p.kproj_fp8) return p.r == 16 ? launch_topm_t<16, true>(p, stream, a, b) : launch_topm_t<32, true>(p, stream, a, b);
+  return p.r == 16 ? launch_topm_t<16, false>(p, stream, a, b) : launch_topm_t<32, false>(p, stream, a, b);
 }
 
 template <int R, bool FP8>

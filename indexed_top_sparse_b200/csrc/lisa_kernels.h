@@ -70,6 +70,24 @@ size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
+// Launch with programmatic stream serialization (the kernel must call pdl_wait before it touches
+// memory an earlier kernel of the stream may write).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // after_sample / after_stream: optional events recorded between the three kernels (nullptr: none).
 cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample = nullptr,
                               cudaEvent_t after_stream = nullptr);

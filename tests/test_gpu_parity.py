@@ -386,13 +386,14 @@ def test_fused_topm_candidate_overflow_falls_back_exactly(cuda_device):
 
 
 def test_fused_topm_too_few_candidates_falls_back_exactly(cuda_device):
-    # High scores only on a few hundred of the positions the threshold sample looks at: the sampled
-    # threshold then sits above the M-th score, fewer than M candidates arrive, and the exact path runs.
+    # High scores only on a few hundred of the positions the threshold sample looks at (runs of 8
+    # adjacent positions, one run every n / 512 positions): the sampled threshold then sits above the
+    # M-th score, fewer than M candidates arrive, and the exact path runs.
     n, M = 100000, 2048
     prob = small(cuda_device, B=1, Hq=4, Hkv=2, d=64, r=16, M=M, seq_lens=[n], paged=False, kproj_fp8=False,
                  plant=("none",), seed=96)
-    S = min(n, 4096)
-    hot = torch.tensor([(j * n) // S for j in range(300)], dtype=torch.long)
+    runs = 4096 // 8
+    hot = torch.tensor([(j // 8) * n // runs + j % 8 for j in range(300)], dtype=torch.long)
     G = prob.G
     for h in range(prob.Hkv):
         qbar = prob.q[0, h * G : (h + 1) * G].double().mean(0)
