@@ -590,7 +590,15 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
     const uint4* c4 = reinterpret_cast<const uint4*>(cand);
     uint4* s4 = reinterpret_cast<uint4*>(cstage);
     const uint32_t npairs = (cnt + 1u) >> 1;  // the buffer capacity is even: the pad pair is readable
-    for (uint32_t i = tid; i < npairs; i += THREADS) s4[i] = __ldcg(c4 + i);
+    for (uint32_t i0 = tid; i0 < npairs; i0 += 4u * THREADS) {  // four 16-byte loads in flight
+      uint4 e[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (i0 + k * THREADS < npairs) e[k] = __ldcg(c4 + i0 + k * THREADS);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (i0 + k * THREADS < npairs) s4[i0 + k * THREADS] = e[k];
+    }
   }
   __syncthreads();
   // Visit (key, position) of every candidate -- or, on the exact fallback, of every position.
@@ -665,53 +673,82 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
   find_digit(v2, need, scan, digit);
   const uint32_t K = (p22 << 10) | digit[0];  // the M-th largest key
   const uint32_t tie_take = digit[1];         // keys equal to K to keep, lowest positions first
+  const bool all_ties = hist[digit[0]] == tie_take;  // usually: every key equal to K is kept
   for_each([&](uint32_t k, uint32_t pos) {
-    if (k > K)
+    if (k > K || (all_ties && k == K))
       atomicOr(&sel[pos >> 5], 1u << (pos & 31));
     else if (k == K)
       atomicOr(&tie[pos >> 5], 1u << (pos & 31));
   });
   __syncthreads();
-  // Keep the tie_take lowest tied positions; then emit every kept position in ascending order.
-  const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
-  const int wb = tid * wpt, we = min(nwords, wb + wpt);
-  uint32_t mine = 0;
-  for (int i = wb; i < we; ++i) mine += __popc(tie[i]);
-  uint32_t rank = block_exclusive_scan(mine, scan, nullptr);
-  for (int i = wb; i < we && rank < tie_take; ++i) {
-    uint32_t bits = tie[i];
-    while (bits && rank < tie_take) {
-      const uint32_t low = bits & (~bits + 1u);
-      sel[i] |= low;
-      bits ^= low;
-      ++rank;
+  if (!all_ties) {
+    // Keep the tie_take lowest tied positions (thread-contiguous words, ascending).
+    const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
+    const int wb = tid * wpt, we = min(nwords, wb + wpt);
+    uint32_t mine = 0;
+    for (int i = wb; i < we; ++i) mine += __popc(tie[i]);
+    uint32_t rank = block_exclusive_scan(mine, scan, nullptr);
+    for (int i = wb; i < we && rank < tie_take; ++i) {
+      uint32_t bits = tie[i];
+      while (bits && rank < tie_take) {
+        const uint32_t low = bits & (~bits + 1u);
+        sel[i] |= low;
+        bits ^= low;
+        ++rank;
+      }
     }
+    __syncthreads();
   }
-  mine = 0;
-  for (int i = wb; i < we; ++i) mine += __popc(sel[i]);
-  uint32_t slot = block_exclusive_scan(mine, scan, nullptr);
-  for (int i = wb; i < we; ++i) {
-    uint32_t bits = sel[i];
-    while (bits) {
-      const int bit = __ffs(bits) - 1;
-      bits &= bits - 1;
-      if (slot < (uint32_t)p.M) idx_out[slot] = i * 32 + bit;
-      ++slot;
+  // Emit every kept position in ascending order.  Warp w owns a contiguous run of words; lane l
+  // reads words l, l + 32, ... of it (no bank conflicts) and a warp scan orders the lanes.
+  {
+    const int lane = tid & 31, warp = tid >> 5, nwarps = THREADS / 32;
+    const int wpw = ((nwords + nwarps - 1) / nwarps + 31) & ~31;  // words per warp
+    const int wb = warp * wpw, we = min(nwords, wb + wpw);
+    uint32_t mine = 0;
+    for (int i = wb + lane; i < we; i += 32) mine += __popc(sel[i]);
+    const uint32_t wtot = __reduce_add_sync(0xffffffffu, mine);
+    if (lane == 0) scan[warp] = wtot;
+    __syncthreads();
+    uint32_t base = 0;
+    for (int w = 0; w < warp; ++w) base += scan[w];
+    for (int i0 = wb; i0 < we; i0 += 32) {
+      const int i = i0 + lane;
+      uint32_t bits = i < we ? sel[i] : 0u;
+      const uint32_t c = __popc(bits);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      uint32_t slot = base + incl - c;
+      while (bits) {
+        const int bit = __ffs(bits) - 1;
+        bits &= bits - 1;
+        if (slot < (uint32_t)p.M) idx_out[slot] = i * 32 + bit;
+        ++slot;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
   if (tid == 0) p.count[bh] = p.M;
 }
 
-constexpr int kStreamChunk = 4096;        // positions per streaming CTA (kStreamChunk / 8 per warp)
+constexpr int kStreamChunk = 4096;        // positions per streaming CTA
 constexpr int kStreamStageBytes = 2048;   // projected-key bytes per warp pipeline stage
 constexpr int kStreamStages = 4;          // stages in each warp's shared-memory ring
+constexpr int kStreamThreads = 128;       // threads of a streaming CTA (4 warps, 1024 positions each)
+constexpr int kStreamCtasPerSm = 5;       // resident streaming CTAs per SM (shared memory bound)
 
-// Each warp streams its own contiguous eighth of the CTA's chunk through a private cp.async ring:
+// Each warp streams its own contiguous quarter of the CTA's chunk through a private cp.async ring:
 // a lane waits only for its own copies and the warp synchronises with __syncwarp, so the streaming
 // loop has no CTA-wide barrier.  Stage s of a warp holds rows [s * RPS, (s + 1) * RPS) of its range
-// (16-byte chunks XOR-swizzled within each row so that the row reads are free of bank conflicts).
+// (for fp32 rows, 16-byte chunks XOR-swizzled within each row so that the row reads are free of
+// bank conflicts).  Positions whose key reaches the threshold are staged in shared memory (one
+// shared atomic per lane that has any) and appended to the pair's candidate buffer at the end.
 template <int R, bool FP8>
-__global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(IndexParams p) {
+__global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_stream_kernel(IndexParams p) {
   extern __shared__ __align__(128) uint8_t ring[];  // [warp][kStreamStages][kStreamStageBytes]
   __shared__ const uint8_t* pbase[kStreamChunk / 16];  // global address of each page block of the chunk
   __shared__ uint32_t ckey[kStageCap];
@@ -722,7 +759,7 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
   constexpr int CPR = RB / 16;                            // 16-byte chunks per row
   constexpr int RPS = kStreamStageBytes / RB;             // rows per stage
   constexpr int RPL = RPS >= 32 ? RPS / 32 : 1;           // rows per lane per stage
-  constexpr int WARPS = kIndexThreads / 32;
+  constexpr int WARPS = kStreamThreads / 32;
   constexpr int WROWS = kStreamChunk / WARPS;             // rows per warp
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -759,6 +796,18 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
   auto issue = [&](int stage) {
     if (stage >= nstages) return;
     uint8_t* dst = wring + (stage % kStreamStages) * kStreamStageBytes;
+    if (FP8 && p.ps >= RPS) {
+      // the stage's rows are contiguous inside one page block: one base, unswizzled 16-byte chunks
+      const int lr0 = w0 + stage * RPS;
+      const uint8_t* base = pbase[lr0 >> p.log2ps] + (lr0 & (p.ps - 1)) * RB;
+      const int vbytes = min(RPS, wrows - stage * RPS) * RB;
+#pragma unroll
+      for (int k = 0; k < kStreamStageBytes / 512; ++k) {
+        const int off = (lane + 32 * k) * 16;
+        cp_async_16(smem_u32(dst + off), base + (off < vbytes ? off : 0), off < vbytes ? 16u : 0u);
+      }
+      return;
+    }
 #pragma unroll
     for (int k = 0; k < kStreamStageBytes / 512; ++k) {
       const int c = lane + 32 * k;  // 16-byte chunk of the stage
@@ -781,7 +830,7 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
   pdl_trigger();
   const uint32_t tau = p.tau[bh];
   const float scale = p.kproj_scale[h];
-  constexpr int NK = FP8 ? 2 * (RPS / 64) : RPL;  // rows a lane keys per stage
+  constexpr int NK = FP8 ? 2 * ((RPS / 16 + 3) / 4) : RPL;  // rows a lane keys per stage
   float2 u2[FP8 ? 1 : R / 2];
   MmaScore<R> mma_score;
   if constexpr (FP8)
@@ -805,11 +854,11 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
       for (int mt = 0; mt < MT; ++mt) mma_score.tile(src + mt * 16 * RB, lane, d[mt]);
       const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-      for (int o = 0; o < MT / 4; ++o) {
+      for (int o = 0; o < (MT + 3) / 4; ++o) {
         float s0 = d[4 * o][0] + d[4 * o][1], s1 = d[4 * o][2] + d[4 * o][3];
 #pragma unroll
         for (int q = 1; q < 4; ++q) {
-          if (t == q) {
+          if (4 * o + q < MT && t == q) {
             s0 = d[4 * o + q][0] + d[4 * o + q][1];
             s1 = d[4 * o + q][2] + d[4 * o + q][3];
           }
@@ -821,7 +870,7 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
       }
 #pragma unroll
       for (int k = 0; k < NK; ++k)
-        if (st * RPS + rloc[k] < wrows && key[k] >= tau) mask |= 1u << k;
+        if (rloc[k] < RPS && st * RPS + rloc[k] < wrows && key[k] >= tau) mask |= 1u << k;
     } else {
 #pragma unroll
       for (int k = 0; k < NK; ++k) {
@@ -840,17 +889,8 @@ __global__ void __launch_bounds__(kIndexThreads, 3) lisa_index_stream_kernel(Ind
         if (r < RPS && st * RPS + r < wrows && key[k] >= tau) mask |= 1u << k;
       }
     }
-    if (__ballot_sync(0xffffffffu, mask != 0u)) {
-      const uint32_t mine = __popc(mask);
-      uint32_t incl = mine;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      uint32_t slot = 0u;
-      if (lane == 31) slot = atomicAdd(&s_ncand, incl);
-      slot = __shfl_sync(0xffffffffu, slot, 31) + incl - mine;
+    if (mask != 0u) {  // a few lanes per stage: one shared-memory atomic each
+      uint32_t slot = atomicAdd(&s_ncand, (uint32_t)__popc(mask));
 #pragma unroll
       for (int k = 0; k < NK; ++k) {
         if ((mask >> k) & 1u) {
@@ -1161,11 +1201,11 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
   if (e != cudaSuccess) return e;
   if (after_sample != nullptr && (e = cudaEventRecord(after_sample, stream)) != cudaSuccess) return e;
   const dim3 grid((p.max_seq_len + kStreamChunk - 1) / kStreamChunk, p.Hkv, p.B);
-  const size_t ring = (size_t)(kIndexThreads / 32) * kStreamStages * kStreamStageBytes;
+  const size_t ring = (size_t)(kStreamThreads / 32) * kStreamStages * kStreamStageBytes;
   auto k = lisa_index_stream_kernel<R, FP8>;
   e = set_smem(k, ring);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(k, grid, dim3(kIndexThreads), ring, stream, p);
+  e = launch_pdl(k, grid, dim3(kStreamThreads), ring, stream, p);
   if (e != cudaSuccess) return e;
   if (after_stream != nullptr && (e = cudaEventRecord(after_stream, stream)) != cudaSuccess) return e;
   const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap);
