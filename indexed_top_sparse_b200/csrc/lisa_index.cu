@@ -410,11 +410,13 @@ constexpr int kSampleThreads = 512;
 constexpr int kSampleRun = 8;  // adjacent positions per sampled run (one 256-byte read at r = 32 FP8)
 
 // Position of sample j of S (S = min(n, kSampleMax)): every position when n <= kSampleMax, else runs
-// of kSampleRun adjacent positions, one run starting every n / (S / kSampleRun) positions.  Runs keep
-// the DRAM reads few and whole-sector; the threshold only needs a rough quantile.
-__device__ __forceinline__ int sample_pos(int j, int n, int S) {
+// of kSampleRun adjacent positions, one run starting every n / (kSampleMax / kSampleRun) positions.
+// Runs keep the DRAM reads few and whole-sector; the threshold only needs a rough quantile.
+static_assert(kSampleMax / kSampleRun == 512, "the run start below divides by 512 with a shift");
+__device__ __forceinline__ int sample_pos(int j, int n) {
   if (n <= kSampleMax) return j;
-  return (int)(((long long)(j / kSampleRun) * n) / (S / kSampleRun)) + (j % kSampleRun);
+  // (j / 8) * n < 2^9 * 2^18 (n <= kMaxSeqLen): exact in 32 bits
+  return (int)(((uint32_t)(j / kSampleRun) * (uint32_t)n) >> 9) + (j % kSampleRun);
 }
 
 template <int R, bool FP8>
@@ -456,15 +458,13 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
       prow[w][i] = (j < p.r && c < p.d) ? __ldg(&p.P[((size_t)h * p.r + j) * p.d + c]) : 0.f;
     }
   }
-  int pg[SPT];
+  int pg[SPT], tpos[SPT];
 #pragma unroll
   for (int k = 0; k < SPT; ++k) {
     const int j = tid + k * kSampleThreads;
     pg[k] = 0;
-    if (sampling && j < S) {
-      const int t = sample_pos(j, n, S);
-      pg[k] = p.page_table[(size_t)b * p.max_pages + (t >> p.log2ps)];
-    }
+    tpos[k] = sample_pos(j, n);
+    if (sampling && j < S) pg[k] = p.page_table[(size_t)b * p.max_pages + (tpos[k] >> p.log2ps)];
   }
   for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
   if (tid < p.d) qbar[tid] = qsum / (float)G;
@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
     for (int k = 0; k < KB; ++k) {
       const int j = tid + (k0 + k) * kSampleThreads;
       if (sampling && j < S) {
-        const int t = sample_pos(j, n, S);
+        const int t = tpos[k0 + k];
         int pgk = pg[k0 + k];
         if (pgk < 0 || pgk >= p.num_pages) {
           bad |= LISA_DEVERR_PAGE_ID;
