@@ -289,6 +289,24 @@ def run_ours(args, world, rank, local):
         t = torch.tensor([e2e_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
+    # Append step (the producer side of the caches) on the same workload: the current token's K/V
+    # rows and FP8 projected keys written into the pools, timed on the device.
+    g = torch.Generator().manual_seed(7)
+    k_new = torch.randn(B, prob.Hkv, d, generator=g).to(torch.bfloat16).to(dev)
+    v_new = torch.randn(B, prob.Hkv, d, generator=g).to(torch.bfloat16).to(dev)
+    def append():
+        L.lisa_append_token(desc, None, k_new, v_new, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale, k_arg, v_arg, ws,
+                            stream=stream)
+    for _ in range(3):
+        append()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a0.record(stream)
+    for _ in range(K):
+        append()
+    a1.record(stream)
+    torch.cuda.synchronize(dev)
+    append_us = a0.elapsed_time(a1) / K * 1e3
     flags = L.lisa_check_device_error(ws)
 
     if rank != 0:
@@ -344,6 +362,13 @@ def run_ours(args, world, rank, local):
             "d2h_bytes_per_step": int(out.numel() * 2),
         },
         "gpu_launches": 4 * K,  # sample, stream, finish, attention
+        "append": {
+            "entry": "lisa_append_token",
+            "us_per_call": append_us,
+            "queries_per_s": B * world / (append_us * 1e-6),
+            "bytes_per_call": int(2 * B * prob.Hkv * d * 2 * 2 + prob.P.numel() * 4 + B * prob.Hkv * prob.r),
+            "bound": "latency (a few hundred KB per call)",
+        },
         "clocks": clk.summary(),
         "device_check_flags": flags,
     }

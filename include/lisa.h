@@ -196,6 +196,27 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
                               float* lse, void* ws, size_t ws_bytes,
                               const lisa_stage_events* events, lisa_stream_t stream);
 
+/* Producer side of the decode step (JSSA write-up, "Как JSSA сохраняет порядок токенов": the
+ * projected keys live in an FP8 cache beside the full-size K/V cache).  For every sequence b and
+ * KV head h, the current token's rows are written at position t_b = positions[b] (positions may be
+ * NULL: t_b = seq_lens[b] - 1), page page_table[b][t_b / page_size], slot t_b % page_size:
+ *   k_pool/v_pool row  <- k_new[b][h][0..d), v_new[b][h][0..d)  (bf16, copied bit for bit)
+ *   kproj_pool row     <- c = P_h k_new[b][h], where c_i = (...((P_i0 k_0) + P_i1 k_1) + ...) + P_i,d-1 k_d-1
+ *                         in fp32 with every product and every sum rounded to nearest even (no
+ *                         fused multiply-add), then
+ *                         LISA_KPROJ_FP8_E4M3: the E4M3 code of c_i / kproj_scale[h] (fp32 division,
+ *                         round to nearest even, magnitudes above 448 saturate to 448);
+ *                         LISA_KPROJ_FP32: c_i.
+ * The arithmetic is fixed so that the codes are reproducible bit for bit.  Layouts as in
+ * lisa_fused_decode (kv_row_stride honoured); k_new, v_new bf16 [B][Hkv][d] (16-byte aligned),
+ * P fp32 [Hkv][r][d].  A position outside [0, max_seq_len) or a page id outside [0, num_pages)
+ * sets LISA_DEVERR_INDEX or LISA_DEVERR_PAGE_ID and that (b, h) writes nothing.  Only the error word
+ * of the workspace is used (its size is lisa_workspace_size(desc) all the same). */
+lisa_status lisa_append_token(const lisa_decode_desc* desc, const int32_t* positions, const void* k_new,
+                              const void* v_new, const float* P, void* kproj_pool, lisa_kproj_dtype kproj_dtype,
+                              const float* kproj_scale, void* k_pool, void* v_pool, void* ws, size_t ws_bytes,
+                              lisa_stream_t stream);
+
 /* Synchronise `stream`, read the workspace error word into *flags_out (may be NULL), clear it.
  * Returns LISA_ERR_DEVICE_CHECK if any bit was set, LISA_OK otherwise. */
 lisa_status lisa_check_device_error(void* ws, uint32_t* flags_out, lisa_stream_t stream);

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     StageEvents,
     alloc_workspace,
     linear_branch,
+    lisa_append_token,
     lisa_check_device_error,
     lisa_fused_decode,
     lisa_index_score,

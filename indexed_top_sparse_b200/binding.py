@@ -102,6 +102,7 @@ _sig = {
         [ctypes.POINTER(DecodeDesc), _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P,
          ctypes.POINTER(LinearBranch), _P, _P, _P, _S, ctypes.POINTER(StageEvents), _P],
     ),
+    "lisa_append_token": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _S, _P]),
     "lisa_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
     "lisa_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -267,6 +268,17 @@ def lisa_fused_decode(desc, q, P, kproj_pool, kproj_dtype, kproj_scale, k_pool, 
             None if events is None else ctypes.byref(events), _stream(stream),
         ),
         "lisa_fused_decode",
+    )
+
+
+def lisa_append_token(desc, positions, k_new, v_new, P, kproj_pool, kproj_dtype, kproj_scale, k_pool, v_pool, ws,
+                      stream=None) -> None:
+    _check(
+        _lib.lisa_append_token(
+            ctypes.byref(desc), _ptr(positions), _ptr(k_new), _ptr(v_new), _ptr(P), _ptr(kproj_pool), kproj_dtype,
+            _ptr(kproj_scale), _ptr(k_pool), _ptr(v_pool), _ptr(ws), ws.numel(), _stream(stream),
+        ),
+        "lisa_append_token",
     )
 
 

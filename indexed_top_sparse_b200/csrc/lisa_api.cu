@@ -447,6 +447,49 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
   return LISA_OK;
 }
 
+lisa_status lisa_append_token(const lisa_decode_desc* desc, const int32_t* positions, const void* k_new,
+                              const void* v_new, const float* P, void* kproj_pool, lisa_kproj_dtype kproj_dtype,
+                              const float* kproj_scale, void* k_pool, void* v_pool, void* ws, size_t ws_bytes,
+                              lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  LISA_TRY(check_idx_dim(desc));
+  if (k_new == nullptr || v_new == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr ||
+      k_pool == nullptr || v_pool == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (kproj_dtype != LISA_KPROJ_FP32 && kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned4(P) ||
+      !aligned4(kproj_scale) || !aligned4(kproj_pool) || (positions != nullptr && !aligned4(positions)))
+    return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  AppendParams p{};
+  p.B = desc->batch;
+  p.Hkv = desc->num_kv_heads;
+  p.d = desc->head_dim;
+  p.r = desc->idx_dim;
+  p.ps = desc->page_size;
+  p.log2ps = ilog2(desc->page_size);
+  p.max_pages = desc->max_pages_per_seq;
+  p.max_seq_len = desc->max_seq_len;
+  p.num_pages = desc->num_pages;
+  p.kv_stride_bytes = (desc->kv_row_stride > 0 ? desc->kv_row_stride : desc->head_dim) * 2;
+  p.kproj_fp8 = kproj_dtype == LISA_KPROJ_FP8_E4M3;
+  p.positions = positions;
+  p.seq_lens = desc->seq_lens;
+  p.page_table = desc->page_table;
+  p.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  p.P = P;
+  p.kproj_scale = kproj_scale;
+  p.kproj = kproj_pool;
+  p.k_pool = static_cast<uint8_t*>(k_pool);
+  p.v_pool = static_cast<uint8_t*>(v_pool);
+  p.err = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_append(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 lisa_status lisa_check_device_error(void* ws, uint32_t* flags_out, lisa_stream_t stream) {
   if (ws == nullptr) return LISA_ERR_WORKSPACE;
   LISA_TRY(bind_device(ws));

@@ -35,6 +35,23 @@ struct IndexParams {
   uint32_t* err;
 };
 
+struct AppendParams {
+  int B, Hkv, d, r, ps, log2ps, max_pages, max_seq_len, num_pages;
+  int kv_stride_bytes;  // bytes between consecutive (page, slot, KV head) rows of the K/V pools
+  bool kproj_fp8;
+  const int32_t* positions;  // [B] or nullptr (seq_lens[b] - 1)
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  const __nv_bfloat16* k_new;  // [B][Hkv][d]
+  const __nv_bfloat16* v_new;
+  const float* P;              // [Hkv][r][d]
+  const float* kproj_scale;    // [Hkv]
+  void* kproj;                 // [num_pages][Hkv][ps][r] of E4M3 codes or fp32
+  uint8_t* k_pool;
+  uint8_t* v_pool;
+  uint32_t* err;
+};
+
 struct AttnParams {
   int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
   int kv_stride_bytes;  // bytes between consecutive (page, slot, KV head) rows of the K/V pools
@@ -93,5 +110,6 @@ cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEve
                               cudaEvent_t after_stream = nullptr);
 size_t finish_smem_bytes(int max_seq_len, int cap);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
 }  // namespace lisa

@@ -256,3 +256,77 @@ def layered_decode(layers: list, full_layers, heads=None) -> list:
             res = decode_step(inp, reuse_idx=last_full, heads=heads)
         results.append(res)
     return results
+
+
+# ---------------------------------------------------------------------------
+# Append: the producer side of the caches (JSSA, "Как JSSA сохраняет порядок
+# токенов": every cached position keeps a projected key in an FP8 cache beside
+# the full-size keys and values)
+# ---------------------------------------------------------------------------
+
+# Non-negative finite E4M3 magnitudes in code order 0x00..0x7E (ascending).
+_E4M3_MAGNITUDES = e4m3_to_f64(np.arange(0x7F))
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Values -> E4M3 codes (uint8): round to nearest, ties to the code with an even mantissa, and
+    magnitudes of 448 and above saturate to 448 (the "satfinite" conversion of the OCP 8-bit format).
+
+    The sign bit follows the sign of x, so -0.0 and small negatives that round to zero give 0x80.
+    NaN gives 0xFF or 0x7F.  Candidates are the two representable neighbours of |x|.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    i = np.clip(np.searchsorted(_E4M3_MAGNITUDES, a, side="left"), 1, 0x7E)
+    lo, hi = _E4M3_MAGNITUDES[i - 1], _E4M3_MAGNITUDES[i]
+    take_hi = (a - lo > hi - a) | ((a - lo == hi - a) & ((i & 1) == 0))
+    code = np.where(take_hi, i, i - 1)
+    code = np.where(a >= 448.0, 0x7E, code)
+    code = np.where(np.isnan(x), 0x7F, code)
+    code = np.where(np.signbit(x), code | 0x80, code)
+    return code.astype(np.uint8)
+
+
+def project_key_fp32(P_h: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """c = P_h k in the fixed fp32 arithmetic of the append step: c_i starts at 0 and adds
+    P_h[i][j] * k[j] for j = 0, 1, ..., d-1, with every product and every sum rounded to fp32
+    (nearest even) separately.  P_h: [r][d], k: [d] (bf16 values, exact in fp32) -> [r] fp32.
+
+    The pages fix no arithmetic for the projection; because the FP8 code is an integer decided by
+    floating point, the oracle takes it in the same fp32 steps as the kernel.
+    """
+    P32 = np.asarray(P_h, dtype=np.float32)
+    k32 = np.asarray(k, dtype=np.float32)
+    c = np.zeros(P32.shape[0], dtype=np.float32)
+    for j in range(P32.shape[1]):
+        prod = (P32[:, j] * k32[j]).astype(np.float32)
+        c = (c + prod).astype(np.float32)
+    return c
+
+
+def append_token(pools: dict, seq_lens, page_table, k_new_bits, v_new_bits, P, kproj_scale, kproj_fp8: bool,
+                 positions=None) -> dict:
+    """Write the current token of every (sequence b, KV head h) into copies of the caches.
+
+    pools: "k", "v": uint16 bf16 bits [num_pages][ps][Hkv][d]; "kproj": uint8 codes or float32
+    [num_pages][Hkv][ps][r].  k_new_bits/v_new_bits: uint16 [B][Hkv][d].  P: [Hkv][r][d] fp32.
+    Position t_b = positions[b], else seq_lens[b] - 1; row = page_table[b][t // ps], slot t % ps.
+    The K/V rows are copied bit for bit; the projected-key row is project_key_fp32(P_h, k), then
+    for FP8 the code of (c / scale_h) rounded to fp32 and encoded by e4m3_encode.
+    """
+    out = {name: np.array(arr, copy=True) for name, arr in pools.items()}
+    ps = out["k"].shape[1]
+    B, Hkv = np.asarray(k_new_bits).shape[:2]
+    for b in range(B):
+        t = int(positions[b]) if positions is not None else int(seq_lens[b]) - 1
+        page, slot = int(page_table[b][t // ps]), t % ps
+        for h in range(Hkv):
+            out["k"][page, slot, h] = k_new_bits[b][h]
+            out["v"][page, slot, h] = v_new_bits[b][h]
+            c = project_key_fp32(P[h], bf16_to_f64(k_new_bits[b][h]))
+            if kproj_fp8:
+                x = (c / np.float32(kproj_scale[h])).astype(np.float32)
+                out["kproj"][page, h, slot] = e4m3_encode(x)
+            else:
+                out["kproj"][page, h, slot] = c
+    return out

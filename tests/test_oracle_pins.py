@@ -379,6 +379,87 @@ def _expect_failure(monkeypatch, name, bad, test_fn, *args):
     monkeypatch.undo()
 
 
+# ---------------------------------------------------------------------------
+# Append step: E4M3 encoder, fixed fp32 projection, cache writes
+# ---------------------------------------------------------------------------
+
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(O.e4m3_encode(O.e4m3_to_f64(codes)), codes)
+
+
+def test_e4m3_encode_matches_library_conversion():
+    # torch's float8_e4m3fn conversion: round to nearest even within the finite range
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(0, 40, 50000), rng.normal(0, 0.01, 20000), rng.uniform(-448, 448, 20000)])
+    x = x.astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x.astype(np.float64)), ref)
+
+
+def test_e4m3_encode_ties_and_saturation():
+    mags = O.e4m3_to_f64(np.arange(0x7F))
+    for c in range(0x7E):  # midpoint between codes c and c + 1 goes to the even one
+        mid = (mags[c] + mags[c + 1]) / 2
+        want = c if c % 2 == 0 else c + 1
+        assert int(O.e4m3_encode(mid)) == want and int(O.e4m3_encode(-mid)) == want | 0x80
+    assert int(O.e4m3_encode(448.0)) == 0x7E and int(O.e4m3_encode(449.0)) == 0x7E
+    assert int(O.e4m3_encode(1e30)) == 0x7E and int(O.e4m3_encode(-1e30)) == 0xFE
+    assert int(O.e4m3_encode(-0.0)) == 0x80 and int(O.e4m3_encode(0.0)) == 0x00
+
+
+def test_fp32_projection_is_sequential_and_within_rounding_of_exact():
+    rng = np.random.default_rng(6)
+    P = rng.normal(0, 1, (32, 128)).astype(np.float32)
+    k = O.bf16_to_f64(_bf16_bits(rng.normal(0, 1, 128)))
+    c = O.project_key_fp32(P, k)
+    exact = P.astype(np.float64) @ k
+    bound = 128 * 2.0**-23 * (np.abs(P.astype(np.float64)) @ np.abs(k))
+    assert np.all(np.abs(c.astype(np.float64) - exact) <= bound)
+    # the fixed order: sequential left-to-right fp32 sums, checked on a case where order matters
+    P2 = np.array([[1.0, 2.0**-24, 2.0**-24, -1.0]], dtype=np.float32)
+    k2 = np.ones(4)
+    assert O.project_key_fp32(P2, k2)[0] == np.float32(0.0)  # (1 + 2^-24) rounds to 1 twice, then - 1
+    # integers are exact in any order
+    P3 = rng.integers(-8, 8, (16, 64)).astype(np.float32)
+    k3 = rng.integers(-8, 8, 64).astype(np.float64)
+    assert np.array_equal(O.project_key_fp32(P3, k3), (P3.astype(np.float64) @ k3).astype(np.float32))
+
+
+def test_append_writes_exactly_the_current_rows():
+    rng = np.random.default_rng(7)
+    pages, ps, Hkv, d, r, B = 6, 16, 2, 64, 16, 3
+    pools = {"k": rng.integers(0, 65535, (pages, ps, Hkv, d)).astype(np.uint16),
+             "v": rng.integers(0, 65535, (pages, ps, Hkv, d)).astype(np.uint16),
+             "kproj": rng.integers(0, 255, (pages, Hkv, ps, r)).astype(np.uint8)}
+    seq_lens = [20, 1, 33]
+    page_table = [[4, 1, 0], [5, 2, 3], [2, 0, 3]]
+    kb = _bf16_bits(rng.normal(0, 1, (B, Hkv, d)))
+    vb = _bf16_bits(rng.normal(0, 1, (B, Hkv, d)))
+    P = rng.normal(0, 1, (Hkv, r, d)).astype(np.float32)
+    scale = np.array([0.05, 0.02], dtype=np.float32)
+    out = O.append_token(pools, seq_lens, page_table, kb, vb, P, scale, True)
+    touched = {(page_table[b][(seq_lens[b] - 1) // ps], (seq_lens[b] - 1) % ps) for b in range(B)}
+    for page in range(pages):
+        for slot in range(ps):
+            same = (page, slot) not in touched
+            assert np.array_equal(out["k"][page, slot], pools["k"][page, slot]) == same
+            assert np.array_equal(out["kproj"][page, :, slot], pools["kproj"][page, :, slot]) == same
+    b = 2  # position 32 -> page_table[2][2] = 3, slot 0
+    assert np.array_equal(out["k"][3, 0], kb[b]) and np.array_equal(out["v"][3, 0], vb[b])
+    for h in range(Hkv):
+        x = (P[h].astype(np.float64) @ O.bf16_to_f64(kb[b][h])) / scale[h]
+        dec = O.e4m3_to_f64(out["kproj"][3, h, 0])
+        sat = np.abs(x) >= 448
+        assert np.all(dec[sat] == np.sign(x[sat]) * 448)  # saturated to the largest finite magnitude
+        # otherwise within half an E4M3 step (2^-4 relative, 2^-10 absolute among subnormals)
+        assert np.all(np.abs(dec - x)[~sat] <= np.maximum(np.abs(x) * 2.0**-4, 2.0**-10)[~sat] * 1.001)
+        assert sat.any() or h == 0
+    out2 = O.append_token(pools, seq_lens, page_table, kb, vb, P, scale, True, positions=[0, 0, 0])
+    assert np.array_equal(out2["k"][4, 0], kb[0]) and np.array_equal(out2["k"][2, 0], kb[2])
+
+
 def test_mutations_are_caught(monkeypatch):
     good_project, good_select, good_attn = O.project_query, O.select_top_m, O.sparse_attention
     good_gate, good_upd = O.gate_combine, O.linear_state_update
@@ -410,4 +491,20 @@ def test_mutations_are_caught(monkeypatch):
     # linear read before the update (current token missing)
     _expect_failure(monkeypatch, "linear_state_update", lambda S, z, k, v: (S, z),
                     test_hand_worked_decode_step_with_linear_branch)
+    # encoder: ties away from zero instead of to even
+    good_enc = O.e4m3_encode
+    def enc_ties_up(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        i = np.clip(np.searchsorted(O._E4M3_MAGNITUDES, a, side="left"), 1, 0x7E)
+        lo, hi = O._E4M3_MAGNITUDES[i - 1], O._E4M3_MAGNITUDES[i]
+        code = np.where(a - lo >= hi - a, i, i - 1)
+        code = np.where(a >= 448.0, 0x7E, code)
+        return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)
+    _expect_failure(monkeypatch, "e4m3_encode", enc_ties_up, test_e4m3_encode_ties_and_saturation)
+    # projection summed in fp64 (order and rounding not the fixed ones)
+    _expect_failure(monkeypatch, "project_key_fp32",
+                    lambda P, k: (np.asarray(P, np.float64) @ np.asarray(k, np.float64)).astype(np.float32),
+                    test_fp32_projection_is_sequential_and_within_rounding_of_exact)
+    assert O.e4m3_encode is good_enc
     assert O.project_query is good_project and O.select_top_m is good_select and O.linear_state_update is good_upd
