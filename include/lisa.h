@@ -196,6 +196,29 @@ lisa_status lisa_fused_decode(const lisa_decode_desc* desc, const void* q, const
                               float* lse, void* ws, size_t ws_bytes,
                               const lisa_stage_events* events, lisa_stream_t stream);
 
+/* ---- Comparators (not on the decode path) --------------------------------------------------
+ * The JSSA write-up states its gain against full attention and against "gather, then attend"
+ * (section "Как JSSA сохраняет порядок токенов").  These two calls make those baselines on the same
+ * GPU with the same kernels, so that the ratios can be measured: */
+
+/* Full attention: every query head over all n_b cached positions (no index).  Same layouts as
+ * lisa_sparse_decode_attn; lse may be NULL.  ws: lisa_dense_workspace_size(desc) bytes, 256-byte
+ * aligned (initialised by lisa_workspace_init).  LISA_ERR_UNSUPPORTED when a (b, KV head) would
+ * need more than 256 partial results (max_seq_len above about 261,000 positions). */
+size_t lisa_dense_workspace_size(const lisa_decode_desc* desc);
+lisa_status lisa_dense_decode_attn(const lisa_decode_desc* desc, const void* q, const void* k_pool,
+                                   const void* v_pool, void* out, float* lse, void* ws, size_t ws_bytes,
+                                   lisa_stream_t stream);
+
+/* Gather of the selected rows into a contiguous buffer: gathered bf16 [B][Hkv][M][2][d] (16-byte
+ * aligned), row i of (b, h) = (K row, V row) of position idx[b][h][i] for i < count[b][h], zeros
+ * after.  Attention over it is lisa_dense_decode_attn on a desc with B*Hkv sequences of one KV head,
+ * n = count, and an identity page table over the buffer.  Only the workspace error word is used
+ * (ws_bytes >= 256); bad indices or page ids are flagged and give zero rows. */
+lisa_status lisa_gather_kv(const lisa_decode_desc* desc, const int32_t* idx, const int32_t* count,
+                           const void* k_pool, const void* v_pool, void* gathered, void* ws, size_t ws_bytes,
+                           lisa_stream_t stream);
+
 /* Producer side of the decode step (JSSA write-up, "Как JSSA сохраняет порядок токенов": the
  * projected keys live in an FP8 cache beside the full-size K/V cache).  For every sequence b and
  * KV head h, the current token's rows are written at position t_b = positions[b] (positions may be

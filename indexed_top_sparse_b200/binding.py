@@ -103,6 +103,9 @@ _sig = {
          ctypes.POINTER(LinearBranch), _P, _P, _P, _S, ctypes.POINTER(StageEvents), _P],
     ),
     "lisa_append_token": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _S, _P]),
+    "lisa_dense_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(DecodeDesc)]),
+    "lisa_dense_decode_attn": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
+    "lisa_gather_kv": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
     "lisa_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
     "lisa_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -279,6 +282,36 @@ def lisa_append_token(desc, positions, k_new, v_new, P, kproj_pool, kproj_dtype,
             _ptr(kproj_scale), _ptr(k_pool), _ptr(v_pool), _ptr(ws), ws.numel(), _stream(stream),
         ),
         "lisa_append_token",
+    )
+
+
+def lisa_dense_workspace_size(desc: DecodeDesc) -> int:
+    return int(_lib.lisa_dense_workspace_size(ctypes.byref(desc)))
+
+
+def alloc_dense_workspace(desc: DecodeDesc, device, stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for lisa_dense_decode_attn."""
+    n = lisa_dense_workspace_size(desc)
+    if n == 0:
+        raise LisaError(1, "lisa_dense_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    lisa_workspace_init(ws, stream)
+    return ws
+
+
+def lisa_dense_decode_attn(desc, q, k_pool, v_pool, out, lse, ws, stream=None) -> None:
+    _check(
+        _lib.lisa_dense_decode_attn(ctypes.byref(desc), _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(out), _ptr(lse),
+                                    _ptr(ws), ws.numel(), _stream(stream)),
+        "lisa_dense_decode_attn",
+    )
+
+
+def lisa_gather_kv(desc, idx, count, k_pool, v_pool, gathered, ws, stream=None) -> None:
+    _check(
+        _lib.lisa_gather_kv(ctypes.byref(desc), _ptr(idx), _ptr(count), _ptr(k_pool), _ptr(v_pool), _ptr(gathered),
+                            _ptr(ws), ws.numel(), _stream(stream)),
+        "lisa_gather_kv",
     )
 
 

@@ -99,6 +99,39 @@ Layout layout_of(const lisa_decode_desc& d) {
   return L;
 }
 
+// Workspace of the dense comparator: error word, partition counters and the partials of a stream-K
+// attention over every position (tiles of the whole context instead of the M selected).
+Layout dense_layout_of(const lisa_decode_desc& d) {
+  Layout L;
+  L.G = d.num_q_heads / d.num_kv_heads;
+  L.tpp = (d.max_seq_len + kAttnTile - 1) / kAttnTile;
+  const long long pairs = d.batch > 0 ? (long long)d.batch * d.num_kv_heads : 1;
+  const long long tiles = pairs * L.tpp;
+  long long grid = tiles < kAttnGrid ? tiles : kAttnGrid;
+  if (grid * kAttnMaxTiles < tiles) grid = (tiles + kAttnMaxTiles - 1) / kAttnMaxTiles;
+  // a pair is covered by at most ceil(grid / pairs) + 1 runs; the merge holds 256 partials
+  const long long cap = (long long)(kMaxBudget / kAttnTile - 1) * pairs;
+  if (grid > cap) grid = cap;
+  L.grid = (int)grid;
+  L.splits = (int)((L.grid + pairs - 1) / pairs) + 1;
+  const size_t B = (size_t)d.batch, Hkv = (size_t)d.num_kv_heads;
+  size_t off = kErrBytes;
+  L.off_acount = off;
+  off += align256(B * Hkv * 4);
+  L.off_opart = off;
+  off += align256(B * Hkv * (size_t)L.splits * L.G * (size_t)d.head_dim * 4);
+  L.off_ml = off;
+  off += align256(B * Hkv * (size_t)L.splits * L.G * 2 * 4);
+  L.total = off;
+  return L;
+}
+
+// Every CTA run holds at most kAttnMaxTiles tiles, and a pair's partials fit the merge (256).
+bool dense_fits_merge(const lisa_decode_desc& d, const Layout& L) {
+  const long long pairs = (long long)d.batch * d.num_kv_heads;
+  return (long long)L.grid * kAttnMaxTiles >= pairs * L.tpp && L.splits <= kMaxBudget / kAttnTile;
+}
+
 lisa_status check_ws(const void* ws, size_t bytes, const Layout& L) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < L.total) return LISA_ERR_WORKSPACE;
   return LISA_OK;
@@ -367,6 +400,60 @@ lisa_status lisa_sparse_decode_attn(const lisa_decode_desc* desc, const void* q,
   LISA_TRY(clear_attn_counters(*desc, L, ws, st));
   return cuda_status(
       launch_sparse_attn(attn_params(*desc, L, ws, q, k_pool, v_pool, idx, count, out, lse, nullptr), st));
+}
+
+size_t lisa_dense_workspace_size(const lisa_decode_desc* desc) {
+  if (check_desc(desc) != LISA_OK) return 0;
+  return dense_layout_of(*desc).total;
+}
+
+lisa_status lisa_dense_decode_attn(const lisa_decode_desc* desc, const void* q, const void* k_pool, const void* v_pool,
+                                   void* out, float* lse, void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  if (q == nullptr || k_pool == nullptr || v_pool == nullptr || out == nullptr) return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned4(q)) return LISA_ERR_INVALID_ARG;
+  const Layout L = dense_layout_of(*desc);
+  if (!dense_fits_merge(*desc, L)) return LISA_ERR_UNSUPPORTED;
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  LISA_TRY(clear_attn_counters(*desc, L, ws, st));
+  AttnParams p = attn_params(*desc, L, ws, q, k_pool, v_pool, nullptr, nullptr, out, lse, nullptr);
+  p.dense = true;
+  p.M = desc->max_seq_len;
+  return cuda_status(launch_sparse_attn(p, st));
+}
+
+lisa_status lisa_gather_kv(const lisa_decode_desc* desc, const int32_t* idx, const int32_t* count, const void* k_pool,
+                           const void* v_pool, void* gathered, void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  if (idx == nullptr || count == nullptr || k_pool == nullptr || v_pool == nullptr || gathered == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(gathered)) return LISA_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < kErrBytes || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return LISA_ERR_WORKSPACE;
+  LISA_TRY(bind_device(ws));
+  GatherParams p{};
+  p.B = desc->batch;
+  p.Hkv = desc->num_kv_heads;
+  p.d = desc->head_dim;
+  p.M = desc->budget_m;
+  p.ps = desc->page_size;
+  p.log2ps = ilog2(desc->page_size);
+  p.max_pages = desc->max_pages_per_seq;
+  p.max_seq_len = desc->max_seq_len;
+  p.num_pages = desc->num_pages;
+  p.kv_stride_bytes = (desc->kv_row_stride > 0 ? desc->kv_row_stride : desc->head_dim) * 2;
+  p.seq_lens = desc->seq_lens;
+  p.page_table = desc->page_table;
+  p.idx = idx;
+  p.count = count;
+  p.k_pool = static_cast<const uint8_t*>(k_pool);
+  p.v_pool = static_cast<const uint8_t*>(v_pool);
+  p.out = static_cast<uint8_t*>(gathered);
+  p.err = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_gather(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_sparse_decode_attn_noalloc(const lisa_decode_desc* desc, const void* q, const void* k_pool,

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   if (tid < npr) {
     const int pr = pr_first + tid, b = pr / p.Hkv;
     int n = p.seq_lens[b];
-    int cnt = p.count[pr];
+    int cnt = p.dense ? min(max(n, 0), p.max_seq_len) : p.count[pr];
     if (n < 0 || n > p.max_seq_len) {
       bad |= LISA_DEVERR_SEQ_LEN;
       n = n < 0 ? 0 : p.max_seq_len;
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
     tpos[k] = 0;
     if (i < ntile) {
       const int gt = t_lo + i, pr = gt / p.tpp, pos = (gt - pr * p.tpp) * kAttnTile + (e % kAttnTile);
-      tpos[k] = __ldg(&p.idx[(size_t)pr * p.M + min(pos, p.M - 1)]);
+      tpos[k] = p.dense ? pos : __ldg(&p.idx[(size_t)pr * p.M + min(pos, p.M - 1)]);
     }
   }
   __syncthreads();

@@ -52,6 +52,18 @@ struct AppendParams {
   uint32_t* err;
 };
 
+struct GatherParams {
+  int B, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages, kv_stride_bytes;
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  const int32_t* idx;    // [B][Hkv][M]
+  const int32_t* count;  // [B][Hkv]
+  const uint8_t* k_pool;
+  const uint8_t* v_pool;
+  uint8_t* out;          // [B][Hkv][M][2][d] bf16: K then V of each selected position
+  uint32_t* err;
+};
+
 struct AttnParams {
   int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
   int kv_stride_bytes;  // bytes between consecutive (page, slot, KV head) rows of the K/V pools
@@ -59,6 +71,7 @@ struct AttnParams {
   int tpp;      // 64-position tiles per pair: ceil(M / 64)
   int grid;     // CTAs of the stream-K launch (<= npairs * tpp)
   int max_seg;  // partial slots per pair: ceil(grid / npairs) + 1
+  bool dense;   // every position t < n_b, in order (M = max_seq_len; idx and count unused)
   float scale_log2;  // softmax scale * log2(e)
   const int32_t* seq_lens;
   const int32_t* page_table;
@@ -110,6 +123,7 @@ cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEve
                               cudaEvent_t after_stream = nullptr);
 size_t finish_smem_bytes(int max_seq_len, int cap);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
+cudaError_t launch_gather(const GatherParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
 }  // namespace lisa

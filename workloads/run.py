@@ -92,3 +92,49 @@ def fused(prob: DecodeProblem, ws: torch.Tensor, desc=None, reuse: Optional[tupl
     L.lisa_fused_decode(desc, prob.q, prob.P, prob.kproj, kproj_dtype(prob), scale, k, v, ridx,
                         rcount, idx, count, lb, out, lse, ws, events=events, stream=stream)
     return {"out": out, "lse": lse, "idx": idx, "count": count}
+
+
+# ---- comparators (not on the decode path) ----
+
+def dense_attention(prob: DecodeProblem, desc=None):
+    """lisa_dense_decode_attn: every query head over all n_b positions."""
+    desc = desc or desc_of(prob)
+    ws = L.alloc_dense_workspace(desc, prob.device)
+    out = torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=prob.device)
+    lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=prob.device)
+    k, v = kv_args(prob)
+    L.lisa_dense_decode_attn(desc, prob.q, k, v, out, lse, ws)
+    return out, lse, ws
+
+
+class GatherThenAttend:
+    """The "gather, then attend" baseline: lisa_gather_kv into a contiguous [B*Hkv][M][2][d] buffer,
+    then lisa_dense_decode_attn over it as B*Hkv sequences of one KV head (identity page table)."""
+
+    def __init__(self, prob: DecodeProblem, count: torch.Tensor):
+        if prob.M % 64 != 0:
+            raise ValueError("the gathered buffer is paged in 64-row pages: M must be a multiple of 64")
+        dev = prob.device
+        self.prob = prob
+        self.Bp, self.pages = prob.B * prob.Hkv, prob.M // 64
+        self.gathered = torch.empty(self.Bp, prob.M, 2, prob.d, dtype=torch.bfloat16, device=dev)
+        self.table = torch.arange(self.Bp * self.pages, dtype=torch.int32, device=dev).view(self.Bp, self.pages)
+        self.count = count
+        self.desc = L.make_desc(batch=self.Bp, num_q_heads=prob.G, num_kv_heads=1, head_dim=prob.d, idx_dim=prob.r,
+                                budget_m=prob.M, page_size=64, max_pages_per_seq=self.pages, max_seq_len=prob.M,
+                                num_pages=self.Bp * self.pages, seq_lens=count.view(-1), page_table=self.table,
+                                softmax_scale=prob.softmax_scale, kv_row_stride=2 * prob.d)
+        self.ws_gather = L.alloc_workspace(desc_of(prob), dev)
+        self.ws_attn = L.alloc_dense_workspace(self.desc, dev)
+        self.out = torch.empty(prob.B, prob.Hq, prob.d, dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty(prob.B, prob.Hq, dtype=torch.float32, device=dev)
+
+    def gather(self, idx: torch.Tensor, stream=None):
+        k, v = kv_args(self.prob)
+        L.lisa_gather_kv(desc_of(self.prob), idx, self.count, k, v, self.gathered, self.ws_gather, stream=stream)
+
+    def attend(self, stream=None):
+        v = L.DevicePtr(self.gathered.data_ptr() + self.prob.d * 2)
+        L.lisa_dense_decode_attn(self.desc, self.prob.q, self.gathered, v, self.out, self.lse, self.ws_attn,
+                                 stream=stream)
+        return self.out, self.lse
