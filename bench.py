@@ -332,6 +332,24 @@ def run_ours(args, world, rank, local):
     inplace_ms = dev_time(lambda: L.lisa_sparse_decode_attn(desc, prob.q, k_arg, v_arg, idx_c, cnt_c, out, lse, ws,
                                                             stream=stream), max(3, min(K, 50)))
     del gta, dense_ws
+    # Multi-query indexer (speculative decoding with 4 draft tokens per sequence): the scores of all
+    # positions for every token, the 4 projected queries forming one tensor-core contraction.
+    Tq = 4
+    qt = torch.randn(B, Tq, prob.Hq, d, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16).to(dev)
+    kproj_bytes_total = float(sum(int(n) * prob.r * prob.Hkv for n in prob.seq_lens.tolist()))
+    mq_scores = torch.empty(B, Tq, prob.Hkv, prob.max_seq_len, dtype=torch.float32, device=dev)
+    mq_ms = dev_time(lambda: L.lisa_index_score_multi(desc, Tq, qt, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale,
+                                                      mq_scores, ws, stream=stream), max(3, min(K, 20)))
+    mq_bytes = float(kproj_bytes_total + mq_scores.numel() * 4)
+    del mq_scores
+    # Basis calibration (once per layer and KV head, off the decode path): 4096 query and 4096 key
+    # samples per KV head of this workload's shape.
+    g2 = torch.Generator().manual_seed(9)
+    cal_q = torch.randn(prob.Hkv, 4096, d, generator=g2).to(torch.bfloat16).to(dev)
+    cal_k = torch.randn(prob.Hkv, 4096, d, generator=g2).to(torch.bfloat16).to(dev)
+    cal_P = torch.empty(prob.Hkv, prob.r, d, dtype=torch.float32, device=dev)
+    cal_ws = torch.zeros(L.lisa_calibrate_workspace_size(prob.Hkv, d), dtype=torch.uint8, device=dev)
+    calib_ms = dev_time(lambda: L.lisa_calibrate_basis(cal_q, cal_k, cal_P, None, cal_ws, stream=stream), 3)
     flags = L.lisa_check_device_error(ws)
 
     if rank != 0:
@@ -396,6 +414,20 @@ def run_ours(args, world, rank, local):
             "gather_share_of_gather_then_attend": gather_ms / (gather_ms + attend_ms),
             "in_place_attention_ms": inplace_ms,
             "gather_then_attend_over_in_place": (gather_ms + attend_ms) / inplace_ms,
+        },
+        "multi_query_index_scores": {
+            "entry": "lisa_index_score_multi",
+            "tokens_per_sequence": Tq,
+            "ms_per_call": mq_ms,
+            "bytes_per_call": mq_bytes,
+            "achieved_gbs": mq_bytes / (mq_ms * 1e-3) / 1e9,
+            "note": "projected keys read once for all tokens; fp32 scores of every visible position written",
+        },
+        "calibration": {
+            "entry": "lisa_calibrate_basis",
+            "ms_per_call": calib_ms,
+            "kv_heads": prob.Hkv,
+            "samples_per_head": "4096 queries + 4096 keys",
         },
         "append": {
             "entry": "lisa_append_token",

@@ -150,6 +150,18 @@ lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const 
                              const float* kproj_scale, float* scores, void* ws, size_t ws_bytes,
                              lisa_stream_t stream);
 
+/* Steps 1-3 for T query tokens per sequence (speculative or chunked decode; 1 <= T <= 8).  q is
+ * bf16 [B][T][Hq][d], token j of sequence b seeing positions t <= n_b - T + j.  Writes
+ * s_t = scale_h <P_h qbar_{b,j,h}, c_t> to scores[b][j][h][t] for those t (later entries are not
+ * written); scores fp32 [B][T][Hkv][max_seq_len].  FP8 projected keys only.  The T projected queries
+ * of a KV head form the N side of one tensor-core contraction per 16-position tile (E4M3 -> f16 is
+ * exact; each query as an f16 hi/lo pair, fp32 accumulation), so the scores agree with an fp32 dot
+ * product to rounding.  Top-M per token: lisa_topm_select on a desc with B*T sequences (b*T + j,
+ * length n_b - T + j + 1) over the same scores buffer. */
+lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens, const void* q, const float* P,
+                                   const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
+                                   float* scores, void* ws, size_t ws_bytes, lisa_stream_t stream);
+
 /* Step 4 from caller-given fp32 scores: idx[b][h][0..count) ascending, count = min(M, n_b),
  * idx[b][h][count..M) = -1. */
 lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx,
@@ -218,6 +230,22 @@ lisa_status lisa_dense_decode_attn(const lisa_decode_desc* desc, const void* q, 
 lisa_status lisa_gather_kv(const lisa_decode_desc* desc, const int32_t* idx, const int32_t* count,
                            const void* k_pool, const void* v_pool, void* gathered, void* ws, size_t ws_bytes,
                            lisa_stream_t stream);
+
+/* ---- Basis calibration (once per layer and KV head, off the decode path) -------------------------
+ * JSSA write-up, "Как JSSA сохраняет порядок токенов": query and key statistics are collected once
+ * and the basis is taken from eigenvectors of a matrix; the subspace is meant to preserve the
+ * query-key scores.  The pages name no matrix; this library's reading: with Q = mean q q^T over the
+ * averaged group queries and K = mean k k^T over the keys of head h, P_h's rows are the top-r
+ * eigenvectors (largest eigenvalue first) of C = (Q K + K Q) / 2 -- the rank-r subspace that
+ * maximises E[(q . k)(q . P^T P k)] = tr(P^T P K Q) -- each row signed so that its entry of largest
+ * magnitude is positive.  q_samples bf16 [Hkv][nq][d], k_samples bf16 [Hkv][nk][d]; P_out fp32
+ * [Hkv][r][d]; eigvals_out fp32 [Hkv][r] or NULL.  d in {64, 128}, r in {16, 32}, nq, nk >= 1.
+ * ws: lisa_calibrate_workspace_size bytes, 256-byte aligned.  fp32 arithmetic (second moments,
+ * then a cyclic Jacobi eigen-decomposition in shared memory). */
+size_t lisa_calibrate_workspace_size(int num_kv_heads, int head_dim);
+lisa_status lisa_calibrate_basis(int num_kv_heads, int head_dim, int idx_dim, const void* q_samples, int nq,
+                                 const void* k_samples, int nk, float* P_out, float* eigvals_out, void* ws,
+                                 size_t ws_bytes, lisa_stream_t stream);
 
 /* Producer side of the decode step (JSSA write-up, "Как JSSA сохраняет порядок токенов": the
  * projected keys live in an FP8 cache beside the full-size K/V cache).  For every sequence b and

@@ -22,12 +22,15 @@ from .binding import (  # noqa: F401
     alloc_workspace,
     linear_branch,
     lisa_append_token,
+    lisa_calibrate_basis,
+    lisa_calibrate_workspace_size,
     lisa_check_device_error,
     lisa_dense_decode_attn,
     lisa_dense_workspace_size,
     lisa_fused_decode,
     lisa_gather_kv,
     lisa_index_score,
+    lisa_index_score_multi,
     lisa_index_topm,
     lisa_num_splits,
     lisa_sparse_decode_attn,

@@ -104,6 +104,9 @@ _sig = {
     ),
     "lisa_append_token": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _S, _P]),
     "lisa_dense_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(DecodeDesc)]),
+    "lisa_calibrate_workspace_size": (ctypes.c_size_t, [_I, _I]),
+    "lisa_index_score_multi": (_I, [ctypes.POINTER(DecodeDesc), _I, _P, _P, _P, _I, _P, _P, _P, _S, _P]),
+    "lisa_calibrate_basis": (_I, [_I, _I, _I, _P, _I, _P, _I, _P, _P, _P, _S, _P]),
     "lisa_dense_decode_attn": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
     "lisa_gather_kv": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
     "lisa_check_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -282,6 +285,33 @@ def lisa_append_token(desc, positions, k_new, v_new, P, kproj_pool, kproj_dtype,
             _ptr(kproj_scale), _ptr(k_pool), _ptr(v_pool), _ptr(ws), ws.numel(), _stream(stream),
         ),
         "lisa_append_token",
+    )
+
+
+def lisa_index_score_multi(desc, num_tokens, q, P, kproj_pool, kproj_dtype, kproj_scale, scores, ws,
+                           stream=None) -> None:
+    _check(
+        _lib.lisa_index_score_multi(ctypes.byref(desc), num_tokens, _ptr(q), _ptr(P), _ptr(kproj_pool), kproj_dtype,
+                                    _ptr(kproj_scale), _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)),
+        "lisa_index_score_multi",
+    )
+
+
+def lisa_calibrate_workspace_size(num_kv_heads: int, head_dim: int) -> int:
+    return int(_lib.lisa_calibrate_workspace_size(num_kv_heads, head_dim))
+
+
+def lisa_calibrate_basis(q_samples, k_samples, P_out, eigvals_out=None, ws=None, stream=None) -> None:
+    """q_samples [Hkv][nq][d], k_samples [Hkv][nk][d] bf16; P_out [Hkv][r][d] fp32; eigvals [Hkv][r]."""
+    Hkv, nq, d = q_samples.shape
+    nk = k_samples.shape[1]
+    r = P_out.shape[1]
+    if ws is None:
+        ws = torch.zeros(lisa_calibrate_workspace_size(Hkv, d), dtype=torch.uint8, device=q_samples.device)
+    _check(
+        _lib.lisa_calibrate_basis(Hkv, d, r, _ptr(q_samples), nq, _ptr(k_samples), nk, _ptr(P_out), _ptr(eigvals_out),
+                                  _ptr(ws), ws.numel(), _stream(stream)),
+        "lisa_calibrate_basis",
     )
 
 

@@ -26,7 +26,7 @@ inline int ilog2(int x) {
 struct Layout {
   int G = 0, grid = 0, tpp = 0, splits = 0, chunk_max = 0, cap = 0;  // splits: partial slots per pair
   size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0;
-  size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_done = 0, off_acount = 0, off_cand = 0, total = 0;
+  size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_acount = 0, off_cand = 0, total = 0;
 };
 
 // Host checks shared by every entry point.  Returns LISA_OK for a valid desc (also when B == 0).
@@ -88,8 +88,6 @@ Layout layout_of(const lisa_decode_desc& d) {
   L.off_tau = off;
   off += align256(B * Hkv * 4);
   L.off_ccount = off;
-  off += align256(B * Hkv * 4);
-  L.off_done = off;
   off += align256(B * Hkv * 4);
   L.off_acount = off;
   off += align256(B * Hkv * 4);
@@ -181,7 +179,6 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   p.uq = reinterpret_cast<float*>(w + L.off_uq);
   p.tau = reinterpret_cast<uint32_t*>(w + L.off_tau);
   p.ccount = reinterpret_cast<uint32_t*>(w + L.off_ccount);
-  p.done = reinterpret_cast<uint32_t*>(w + L.off_done);
   p.acount = reinterpret_cast<uint32_t*>(w + L.off_acount);
   p.cand = reinterpret_cast<uint32_t*>(w + L.off_cand);
   return p;
@@ -343,6 +340,43 @@ lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const 
   p.kproj_scale = kproj_scale;
   p.scores = scores;
   return cuda_status(launch_index_score(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens, const void* q, const float* P,
+                                   const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
+                                   float* scores, void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  LISA_TRY(check_idx_dim(desc));
+  if (num_tokens < 1 || num_tokens > 8) return LISA_ERR_UNSUPPORTED;
+  if (kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_UNSUPPORTED;
+  if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || scores == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (!aligned32(kproj_pool) || !aligned4(q) || !aligned4(scores) || !aligned4(P)) return LISA_ERR_INVALID_ARG;
+  const Layout L = layout_of(*desc);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  MultiParams p{};
+  p.B = desc->batch;
+  p.T = num_tokens;
+  p.Hq = desc->num_q_heads;
+  p.Hkv = desc->num_kv_heads;
+  p.d = desc->head_dim;
+  p.r = desc->idx_dim;
+  p.ps = desc->page_size;
+  p.log2ps = ilog2(desc->page_size);
+  p.max_pages = desc->max_pages_per_seq;
+  p.max_seq_len = desc->max_seq_len;
+  p.num_pages = desc->num_pages;
+  p.seq_lens = desc->seq_lens;
+  p.page_table = desc->page_table;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.P = P;
+  p.kproj = kproj_pool;
+  p.kproj_scale = kproj_scale;
+  p.scores = scores;
+  p.err = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_index_score_multi(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx, int32_t* count,
@@ -575,6 +609,40 @@ lisa_status lisa_append_token(const lisa_decode_desc* desc, const int32_t* posit
   p.v_pool = static_cast<uint8_t*>(v_pool);
   p.err = static_cast<uint32_t*>(ws);
   return cuda_status(launch_append(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t lisa_calibrate_workspace_size(int num_kv_heads, int head_dim) {
+  if (num_kv_heads <= 0 || (head_dim != 64 && head_dim != 128)) return 0;
+  return kErrBytes + 2 * align256((size_t)num_kv_heads * head_dim * head_dim * 4);
+}
+
+lisa_status lisa_calibrate_basis(int num_kv_heads, int head_dim, int idx_dim, const void* q_samples, int nq,
+                                 const void* k_samples, int nk, float* P_out, float* eigvals_out, void* ws,
+                                 size_t ws_bytes, lisa_stream_t stream) {
+  if (num_kv_heads <= 0 || num_kv_heads > 65535 || nq <= 0 || nk <= 0) return LISA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LISA_ERR_UNSUPPORTED;
+  if (idx_dim != 16 && idx_dim != 32) return LISA_ERR_UNSUPPORTED;
+  if (q_samples == nullptr || k_samples == nullptr || P_out == nullptr) return LISA_ERR_INVALID_ARG;
+  if (!aligned4(q_samples) || !aligned4(k_samples) || !aligned4(P_out) ||
+      (eigvals_out != nullptr && !aligned4(eigvals_out)))
+    return LISA_ERR_INVALID_ARG;
+  const size_t need = lisa_calibrate_workspace_size(num_kv_heads, head_dim);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < need) return LISA_ERR_WORKSPACE;
+  LISA_TRY(bind_device(ws));
+  CalibParams p{};
+  p.Hkv = num_kv_heads;
+  p.d = head_dim;
+  p.r = idx_dim;
+  p.nq = nq;
+  p.nk = nk;
+  p.q = static_cast<const __nv_bfloat16*>(q_samples);
+  p.k = static_cast<const __nv_bfloat16*>(k_samples);
+  char* w = static_cast<char*>(ws);
+  p.Q = reinterpret_cast<float*>(w + kErrBytes);
+  p.K = reinterpret_cast<float*>(w + kErrBytes + align256((size_t)num_kv_heads * head_dim * head_dim * 4));
+  p.P = P_out;
+  p.eigvals = eigvals_out;
+  return cuda_status(launch_calibrate(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_check_device_error(void* ws, uint32_t* flags_out, lisa_stream_t stream) {

@@ -509,7 +509,6 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   if (tid < p.r) p.uq[bh * 32 + tid] = u[tid];
   if (tid == 0) {
     p.ccount[bh] = 0u;
-    p.done[bh] = 0u;
     p.acount[bh] = 0u;
   }
   if (!sampling) {  // every position is kept; the streaming kernel skips this pair
@@ -918,6 +917,146 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
   }
 }
 
+// Multi-query indexer scores (lisa_index_score_multi): T query tokens per sequence.  Token j of
+// sequence b sees positions t <= n_b - T + j; s[b][j][h][t] = scale_h <P_h qbar_{b,j,h}, c_t>.  The
+// T projected queries of a KV head are the columns of one tensor-core contraction over 16-row tiles
+// of FP8 projected keys: column pair (2j, 2j+1) holds u_j as 2^E_j (hi + lo) in f16, so lane (g, t)
+// of a warp finds query 4 nt + t of n-tile nt for rows g and g + 8 of every tile.  The A fragments
+// are loaded straight from the page blocks (8 consecutive rows of 32 bytes per lane group).
+constexpr int kMultiMaxT = 8;
+constexpr int kMultiChunk = 4096;
+constexpr int kMultiThreads = 128;
+
+template <int R>
+__global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiParams p) {
+  __shared__ float qbar[kMultiMaxT][128];
+  __shared__ float ush[kMultiMaxT][32];
+  __shared__ const uint8_t* pbase[kMultiChunk / 16];
+  constexpr int RB = R;                       // FP8: one byte per dimension
+  constexpr int NT = (2 * kMultiMaxT) / 8;    // n-tiles of 8 columns
+  constexpr int KS = R / 16;                  // k-steps of 16 dimensions
+  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int T = p.T, G = p.Hq / p.Hkv, d = p.d;
+  int n = p.seq_lens[b];
+  if (n < 0 || n > p.max_seq_len) {
+    if (tid == 0) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
+    n = n < 0 ? 0 : p.max_seq_len;
+  }
+  const int t_begin = blockIdx.x * kMultiChunk;
+  if (t_begin >= n) return;
+  const int nrows = min(n - t_begin, kMultiChunk);
+  // Projected queries of the T tokens (every CTA of the pair forms them; they are tiny).
+  for (int e = tid; e < T * d; e += blockDim.x) {
+    const int j = e / d, k = e % d;
+    float acc = 0.f;
+    for (int gg = 0; gg < G; ++gg) acc += __bfloat162float(p.q[(((size_t)b * T + j) * p.Hq + (size_t)h * G + gg) * d + k]);
+    qbar[j][k] = acc / (float)G;
+  }
+  {
+    const int npg = (nrows + p.ps - 1) >> p.log2ps;
+    for (int i = tid; i < npg; i += blockDim.x) {
+      int pid = p.page_table[(size_t)b * p.max_pages + (t_begin >> p.log2ps) + i];
+      if (pid < 0 || pid >= p.num_pages) {
+        flag_error(p.err, LISA_DEVERR_PAGE_ID);
+        pid = 0;
+      }
+      pbase[i] = reinterpret_cast<const uint8_t*>(p.kproj) + ((((size_t)pid * p.Hkv + h) << p.log2ps) * RB);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < T * R; e += blockDim.x) {
+    const int j = e / R, i = e % R;
+    const float* Pr = p.P + ((size_t)h * R + i) * d;
+    float acc = 0.f;
+    for (int k = 0; k < d; ++k) acc = fmaf(Pr[k], qbar[j][k], acc);
+    ush[j][i] = acc;
+  }
+  __syncthreads();
+  // B fragments: lane (g, t4) holds column g of each n-tile, i.e. query (8 nt + g) / 2, part g & 1.
+  uint32_t bf[NT][KS][2];
+  float fac[NT];  // output scale of query 4 nt + t4
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int col = 8 * nt + g, j = col >> 1;
+    float mx = 0.f;
+    if (j < T)
+      for (int i = 0; i < R; ++i) mx = fmaxf(mx, fabsf(ush[j][i]));
+    const int E = mx > 0.f ? ilogbf(mx) - 13 : 0;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int e0 = (R / 4) * t4 + 4 * ks + 2 * jj;
+        __half v[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float x = j < T ? ldexpf(ush[j][e0 + q], -E) : 0.f;
+          const __half hi = __float2half_rn(x);
+          v[q] = (col & 1) ? __float2half_rn(x - __half2float(hi)) : hi;
+        }
+        bf[nt][ks][jj] = (uint32_t)__half_as_ushort(v[0]) | ((uint32_t)__half_as_ushort(v[1]) << 16);
+      }
+    }
+    const int jo = 4 * nt + t4;  // the query whose score this lane receives from n-tile nt
+    float mo = 0.f;
+    if (jo < T)
+      for (int i = 0; i < R; ++i) mo = fmaxf(mo, fabsf(ush[jo][i]));
+    const int Eo = mo > 0.f ? ilogbf(mo) - 13 : 0;
+    fac[nt] = p.kproj_scale[h] * ldexpf(1.f, Eo);
+  }
+  // Each warp scores its quarter of the chunk, 16-row tiles, four tiles per batch of loads.
+  const int wrows = kMultiChunk / 4, w0 = warp * wrows;
+  const int rows_here = max(0, min(nrows - w0, wrows));
+  auto row_ptr = [&](int lr) { return pbase[lr >> p.log2ps] + (lr & (p.ps - 1)) * RB + (RB / 4) * t4; };
+  for (int r0 = 0; r0 < rows_here; r0 += 64) {
+    uint32_t a[4][2][R / 16];  // [tile][row g / g + 8][word]
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int lr = w0 + r0 + 16 * tt + g + 8 * hh;
+        const bool ok = lr < w0 + rows_here;
+        const uint8_t* src = row_ptr(ok ? lr : w0);
+        if constexpr (R == 32) {
+          const uint2 v = ok ? *reinterpret_cast<const uint2*>(src) : make_uint2(0u, 0u);
+          a[tt][hh][0] = v.x;
+          a[tt][hh][1] = v.y;
+        } else {
+          a[tt][hh][0] = ok ? *reinterpret_cast<const uint32_t*>(src) : 0u;
+        }
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 4; ++tt) {
+      float dacc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) dacc[nt][0] = dacc[nt][1] = dacc[nt][2] = dacc[nt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_f16x2(a[tt][0][ks], a0, a2);
+        e4m3x4_to_f16x2(a[tt][1][ks], a1, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_f16_16816(dacc[nt], a0, a1, a2, a3, bf[nt][ks][0], bf[nt][ks][1]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int j = 4 * nt + t4;
+        if (j >= T) continue;
+        const int lim = n - T + j;  // last position token j sees
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int pos = t_begin + w0 + r0 + 16 * tt + g + 8 * hh;
+          if (pos <= lim && pos - t_begin < w0 + rows_here)
+            p.scores[(((size_t)b * T + j) * p.Hkv + h) * p.max_seq_len + pos] =
+                fac[nt] * (dacc[nt][2 * hh] + dacc[nt][2 * hh + 1]);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 size_t select_smem_bytes(int chunk_max, int ps) {
@@ -1226,6 +1365,15 @@ template <int R, bool FP8>
 static cudaError_t launch_score_t(const IndexParams& p, cudaStream_t stream) {
   dim3 grid((p.max_seq_len + kScoreChunk - 1) / kScoreChunk, p.Hkv, p.B);
   lisa_score_kernel<R, FP8><<<grid, kIndexThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream) {
+  const dim3 grid((p.max_seq_len + kMultiChunk - 1) / kMultiChunk, p.Hkv, p.B);
+  if (p.r == 16)
+    lisa_score_multi_kernel<16><<<grid, kMultiThreads, 0, stream>>>(p);
+  else
+    lisa_score_multi_kernel<32><<<grid, kMultiThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -20,7 +20,6 @@ struct IndexParams {
   float* uq;           // [B][Hkv][32]: projected averaged query (written by the sample kernel)
   uint32_t* tau;       // [B][Hkv]: candidate threshold key
   uint32_t* ccount;    // [B][Hkv]: candidates appended (may exceed cap: overflow)
-  uint32_t* done;      // [B][Hkv]: streaming CTAs finished
   uint32_t* acount;    // [B][Hkv]: attention partition counters, zeroed here for the fused path
   uint32_t* cand;      // [B][Hkv][cap][2]: (key, position)
   const int32_t* seq_lens;
@@ -64,6 +63,28 @@ struct GatherParams {
   uint32_t* err;
 };
 
+struct CalibParams {
+  int Hkv, d, r, nq, nk;
+  const __nv_bfloat16* q;  // [Hkv][nq][d] averaged group queries
+  const __nv_bfloat16* k;  // [Hkv][nk][d] keys
+  float* Q;                // [Hkv][d][d] second moments (workspace)
+  float* K;
+  float* P;                // [Hkv][r][d] out
+  float* eigvals;          // [Hkv][r] out, nullable
+};
+
+struct MultiParams {
+  int B, T, Hq, Hkv, d, r, ps, log2ps, max_pages, max_seq_len, num_pages;
+  const int32_t* seq_lens;
+  const int32_t* page_table;
+  const __nv_bfloat16* q;  // [B][T][Hq][d]
+  const float* P;          // [Hkv][r][d]
+  const void* kproj;       // FP8 E4M3 [num_pages][Hkv][ps][r]
+  const float* kproj_scale;
+  float* scores;           // [B][T][Hkv][max_seq_len]
+  uint32_t* err;
+};
+
 struct AttnParams {
   int B, Hq, Hkv, d, M, ps, log2ps, max_pages, max_seq_len, num_pages;
   int kv_stride_bytes;  // bytes between consecutive (page, slot, KV head) rows of the K/V pools
@@ -98,6 +119,7 @@ struct AttnParams {
 
 size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
+cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
 // Launch with programmatic stream serialization (the kernel must call pdl_wait before it touches
@@ -124,6 +146,7 @@ cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEve
 size_t finish_smem_bytes(int max_seq_len, int cap);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_gather(const GatherParams& p, cudaStream_t stream);
+cudaError_t launch_calibrate(const CalibParams& p, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
 }  // namespace lisa

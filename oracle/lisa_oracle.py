@@ -330,3 +330,61 @@ def append_token(pools: dict, seq_lens, page_table, k_new_bits, v_new_bits, P, k
             else:
                 out["kproj"][page, h, slot] = c
     return out
+
+
+# ---------------------------------------------------------------------------
+# Basis calibration (JSSA, "Как JSSA сохраняет порядок токенов": per head and
+# layer, statistics of queries and keys are collected once and the basis is
+# taken from eigenvectors of a matrix; the subspace is meant to preserve the
+# query-key scores, not to reconstruct the vectors)
+# ---------------------------------------------------------------------------
+
+
+def calibration_matrix(q_samples: np.ndarray, k_samples: np.ndarray) -> np.ndarray:
+    """C = (Q K + K Q) / 2 with Q = mean q q^T over the averaged group queries and K = mean k k^T.
+
+    Reading (the pages name no matrix): for independent q and k, the expected product of the true
+    score and the score through the projector Pi = P^T P is E[(q.k)(q.Pi k)] = tr(Pi K Q) =
+    tr(Pi C); the rank-r projector maximising it spans the top-r eigenvectors of C.
+    """
+    q = np.asarray(q_samples, dtype=np.float64)
+    k = np.asarray(k_samples, dtype=np.float64)
+    Q = q.T @ q / q.shape[0]
+    K = k.T @ k / k.shape[0]
+    return 0.5 * (Q @ K + K @ Q)
+
+
+def calibrate_basis(q_samples: np.ndarray, k_samples: np.ndarray, r: int):
+    """P [r][d] (orthonormal rows, largest eigenvalue first) and its eigenvalues [r].
+
+    Each row's sign is fixed so that its entry of largest magnitude is positive.
+    """
+    w, V = np.linalg.eigh(calibration_matrix(q_samples, k_samples))
+    order = np.argsort(w)[::-1][:r]
+    P = V[:, order].T.copy()
+    for i in range(r):
+        j = int(np.argmax(np.abs(P[i])))
+        if P[i, j] < 0:
+            P[i] = -P[i]
+    return P, w[order]
+
+
+# ---------------------------------------------------------------------------
+# Multi-query indexer (several query tokens per sequence, e.g. speculative
+# decoding): the same score per token, each token seeing the positions up to
+# its own (causal)
+# ---------------------------------------------------------------------------
+
+
+def multi_query_scores(inp: dict, q_tokens, T: int, b: int, h: int) -> np.ndarray:
+    """[T][n_b] fp64 indexer scores of the T query tokens q_tokens[b] ([T][Hq][d] bf16 bits) of
+    sequence b for KV head h.  Token j sees positions t <= n_b - T + j; later entries are -inf."""
+    n = int(inp["seq_lens"][b])
+    out = np.full((T, n), -np.inf)
+    for j in range(T):
+        one = dict(inp)
+        one["q"] = np.asarray(q_tokens)[:, j]  # [B][Hq][d]: token j of every sequence
+        s = head_scores(one, b, h)
+        lim = n - T + j
+        out[j, : lim + 1] = s[: lim + 1]
+    return out

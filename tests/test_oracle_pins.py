@@ -460,6 +460,86 @@ def test_append_writes_exactly_the_current_rows():
     assert np.array_equal(out2["k"][4, 0], kb[0]) and np.array_equal(out2["k"][2, 0], kb[2])
 
 
+# ---------------------------------------------------------------------------
+# Basis calibration
+# ---------------------------------------------------------------------------
+
+
+def _orthonormal(rng, r, d):
+    return np.linalg.qr(rng.normal(size=(d, r)))[0].T
+
+
+def test_calibration_with_isotropic_queries_is_key_pca():
+    # Q = I (queries = sqrt(d) times an orthogonal matrix): the basis is the keys' principal subspace,
+    # taken here from the SVD of the key samples
+    rng = np.random.default_rng(8)
+    d, r = 64, 16
+    q = np.sqrt(d) * np.linalg.qr(rng.normal(size=(d, d)))[0]
+    k = rng.normal(size=(3000, d)) * np.linspace(4, 0.2, d)
+    P, _ = O.calibrate_basis(q, k, r)
+    Vt = np.linalg.svd(k, full_matrices=False)[2][:r]
+    assert np.allclose(P.T @ P, Vt.T @ Vt, atol=1e-8)
+
+
+def test_calibration_diagonal_moments_pick_largest_products():
+    d, r = 32, 8
+    a = np.linspace(1, 2, d)[::-1] ** 2
+    b = np.roll(np.linspace(0.5, 3, d), 11) ** 2
+    q = np.diag(np.sqrt(a * d))  # Q = diag(a)
+    k = np.diag(np.sqrt(b * d))  # K = diag(b)
+    P, w = O.calibrate_basis(q, k, r)
+    top = np.argsort(a * b)[::-1][:r]
+    assert np.allclose(np.abs(P), np.eye(d)[top], atol=1e-12) and np.all(P[np.arange(r), top] > 0)
+    assert np.allclose(w, (a * b)[top])
+
+
+def test_calibration_maximises_the_score_agreement():
+    # brute force over all sample pairs: mean of (q.k)(q.P^T P k) equals tr(P C P^T), and the
+    # calibrated basis beats random orthonormal bases on it
+    rng = np.random.default_rng(9)
+    d, r = 32, 6
+    q = rng.normal(size=(300, d)) @ np.diag(np.linspace(2, 0.5, d))
+    k = rng.normal(size=(400, d)) @ np.diag(np.linspace(0.3, 2.5, d))
+    P, w = O.calibrate_basis(q, k, r)
+    def agreement(B):
+        S = q @ k.T
+        Sp = (q @ B.T) @ (B @ k.T)
+        return float(np.mean(S * Sp))
+    C = O.calibration_matrix(q, k)
+    assert np.isclose(agreement(P), np.trace(P @ C @ P.T), rtol=1e-10)
+    assert np.isclose(agreement(P), float(np.sort(np.linalg.eigvalsh(C))[::-1][:r].sum()), rtol=1e-10)
+    best_random = max(agreement(_orthonormal(rng, r, d)) for _ in range(200))
+    assert agreement(P) > best_random
+    assert np.allclose(P @ P.T, np.eye(r), atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Multi-query indexer
+# ---------------------------------------------------------------------------
+
+
+def test_multi_query_scores_are_single_queries_over_causal_prefixes():
+    # token j of T equals a one-token decode of the same sequence cut to n - T + j + 1 positions
+    prob = make_problem(name="mq", B=2, Hq=8, Hkv=2, d=64, r=16, M=16, seq_lens=[300, 40], page_size=16, paged=True,
+                        kproj_fp8=True, plant=("none",), seed=30, device=torch.device("cpu"))
+    inp = host_inputs(prob)
+    T = 3
+    rng = np.random.default_rng(31)
+    qt = _bf16_bits(rng.normal(size=(prob.B, T, prob.Hq, prob.d)))
+    for b in range(prob.B):
+        n = int(inp["seq_lens"][b])
+        for h in range(prob.Hkv):
+            s = O.multi_query_scores(inp, qt, T, b, h)
+            for j in range(T):
+                one = dict(inp)
+                one["q"] = qt[:, j]
+                one["seq_lens"] = np.array(inp["seq_lens"]).copy()
+                one["seq_lens"][b] = n - T + j + 1
+                ref = O.head_scores(one, b, h)
+                assert np.allclose(s[j, : n - T + j + 1], ref, rtol=1e-12, atol=1e-12)
+                assert np.all(np.isneginf(s[j, n - T + j + 1 :]))
+
+
 def test_mutations_are_caught(monkeypatch):
     good_project, good_select, good_attn = O.project_query, O.select_top_m, O.sparse_attention
     good_gate, good_upd = O.gate_combine, O.linear_state_update
@@ -507,4 +587,21 @@ def test_mutations_are_caught(monkeypatch):
                     lambda P, k: (np.asarray(P, np.float64) @ np.asarray(k, np.float64)).astype(np.float32),
                     test_fp32_projection_is_sequential_and_within_rounding_of_exact)
     assert O.e4m3_encode is good_enc
+    # calibration matrix taken from the keys alone (plain key PCA)
+    good_cal = O.calibration_matrix
+    _expect_failure(monkeypatch, "calibration_matrix",
+                    lambda q, k: np.asarray(k, np.float64).T @ np.asarray(k, np.float64) / len(k),
+                    test_calibration_diagonal_moments_pick_largest_products)
+    assert O.calibration_matrix is good_cal
+    # multi-query causal limit off by one (token j seeing one position too few)
+    good_mq = O.multi_query_scores
+    def mq_short(inp, q_tokens, T, b, h):
+        out = good_mq(inp, q_tokens, T, b, h)
+        n = int(inp["seq_lens"][b])
+        for j in range(T):
+            out[j, n - T + j] = -np.inf
+        return out
+    _expect_failure(monkeypatch, "multi_query_scores", mq_short,
+                    test_multi_query_scores_are_single_queries_over_causal_prefixes)
+    assert O.multi_query_scores is good_mq
     assert O.project_query is good_project and O.select_top_m is good_select and O.linear_state_update is good_upd
