@@ -146,6 +146,15 @@ def dist_setup(args):
     return world, rank, local
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def oracle_sample(prob_host_fn, budget_s: float):
     """Time the oracle on whole queries (one sequence, all KV heads) until budget_s is spent."""
     from threadpoolctl import threadpool_limits
@@ -264,10 +273,7 @@ def run_ours(args, world, rank, local):
     finish_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
     idx_ms = sum(e[0].elapsed_time(e[3]) for e in evs) / K
     attn_ms = sum(e[3].elapsed_time(e[5]) for e in evs) / K
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_step = ms / K
 
     # End to end through the same entry point: q from pinned host memory in, out back to pinned host memory.
@@ -285,10 +291,7 @@ def run_ours(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / K2
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     # Append step (the producer side of the caches) on the same workload: the current token's K/V
     # rows and FP8 projected keys written into the pools, timed on the device.
     g = torch.Generator().manual_seed(7)
