@@ -231,10 +231,10 @@ def run_ours(args, world, rank, local):
 
     k_arg, v_arg = R.kv_args(prob)
 
-    def step(events=None, q=None):
+    def step(events=None, q=None, o=None):
         L.lisa_fused_decode(desc, prob.q if q is None else q, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale,
-                            k_arg, v_arg, None, None, None, None, None, out, lse, ws, events=events,
-                            stream=stream)
+                            k_arg, v_arg, None, None, None, None, None, out if o is None else o, lse, ws,
+                            events=events, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -276,18 +276,41 @@ def run_ours(args, world, rank, local):
     ms = max_over_ranks(ms, world, dev)
     ms_step = ms / K
 
-    # End to end through the same entry point: q from pinned host memory in, out back to pinned host memory.
+    # End to end through the same entry point: every step's q comes in from pinned host memory and its
+    # output goes back to pinned host memory.  As a serving loop would, the copies run on their own
+    # streams into double buffers, so step k's copy-out and step k+1's copy-in overlap the kernels.
     q_host = prob.q.cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    q_dev = torch.empty_like(prob.q)
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    q_dev = [torch.empty_like(prob.q) for _ in range(2)]
+    out_dev = [torch.empty_like(out) for _ in range(2)]
+    copy_in, copy_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_step = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for i in range(2):  # create the events
+        ev_step[i].record(stream)
+        ev_out[i].record(stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     K2 = max(1, min(K, 100))
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(K2):
-        q_dev.copy_(q_host, non_blocking=True)
-        step(q=q_dev)
-        out_host.copy_(out, non_blocking=True)
+    copy_in.wait_event(e0)
+    copy_out.wait_event(e0)
+    for k in range(K2):
+        i = k % 2
+        copy_in.wait_event(ev_step[i])  # step k - 2 has finished reading q_dev[i]
+        with torch.cuda.stream(copy_in):
+            q_dev[i].copy_(q_host, non_blocking=True)
+        ev_in[i].record(copy_in)
+        stream.wait_event(ev_in[i])
+        stream.wait_event(ev_out[i])  # out_dev[i] of step k - 2 has been copied out
+        step(q=q_dev[i], o=out_dev[i])
+        ev_step[i].record(stream)
+        copy_out.wait_event(ev_step[i])
+        with torch.cuda.stream(copy_out):
+            out_host[i].copy_(out_dev[i], non_blocking=True)
+        ev_out[i].record(copy_out)
+    stream.wait_event(ev_out[(K2 - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / K2

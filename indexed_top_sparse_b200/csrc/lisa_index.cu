@@ -1009,8 +1009,9 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiPa
   const int wrows = kMultiChunk / 4, w0 = warp * wrows;
   const int rows_here = max(0, min(nrows - w0, wrows));
   auto row_ptr = [&](int lr) { return pbase[lr >> p.log2ps] + (lr & (p.ps - 1)) * RB + (RB / 4) * t4; };
-  for (int r0 = 0; r0 < rows_here; r0 += 64) {
-    uint32_t a[4][2][R / 16];  // [tile][row g / g + 8][word]
+  // Software pipeline: the next 64 rows' fragments are in flight while the current ones are used.
+  uint32_t a[2][4][2][R / 16];  // [buffer][tile][row g / g + 8][word]
+  auto load = [&](int r0, uint32_t (&buf)[4][2][R / 16]) {
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
 #pragma unroll
@@ -1018,15 +1019,18 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiPa
         const int lr = w0 + r0 + 16 * tt + g + 8 * hh;
         const bool ok = lr < w0 + rows_here;
         const uint8_t* src = row_ptr(ok ? lr : w0);
-        if constexpr (R == 32) {
-          const uint2 v = ok ? *reinterpret_cast<const uint2*>(src) : make_uint2(0u, 0u);
-          a[tt][hh][0] = v.x;
-          a[tt][hh][1] = v.y;
+        if constexpr (R == 32) {  // read-only loads: free to move ahead of the score stores
+          const uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0u, 0u);
+          buf[tt][hh][0] = v.x;
+          buf[tt][hh][1] = v.y;
         } else {
-          a[tt][hh][0] = ok ? *reinterpret_cast<const uint32_t*>(src) : 0u;
+          buf[tt][hh][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(src)) : 0u;
         }
       }
     }
+  };
+  float* __restrict__ out_scores = p.scores;
+  auto score = [&](int r0, const uint32_t (&buf)[4][2][R / 16]) {
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt) {
       float dacc[NT][4];
@@ -1035,8 +1039,8 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiPa
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t a0, a1, a2, a3;
-        e4m3x4_to_f16x2(a[tt][0][ks], a0, a2);
-        e4m3x4_to_f16x2(a[tt][1][ks], a1, a3);
+        e4m3x4_to_f16x2(buf[tt][0][ks], a0, a2);
+        e4m3x4_to_f16x2(buf[tt][1][ks], a1, a3);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) mma_f16_16816(dacc[nt], a0, a1, a2, a3, bf[nt][ks][0], bf[nt][ks][1]);
       }
@@ -1049,11 +1053,19 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiPa
         for (int hh = 0; hh < 2; ++hh) {
           const int pos = t_begin + w0 + r0 + 16 * tt + g + 8 * hh;
           if (pos <= lim && pos - t_begin < w0 + rows_here)
-            p.scores[(((size_t)b * T + j) * p.Hkv + h) * p.max_seq_len + pos] =
+            out_scores[(((size_t)b * T + j) * p.Hkv + h) * p.max_seq_len + pos] =
                 fac[nt] * (dacc[nt][2 * hh] + dacc[nt][2 * hh + 1]);
         }
       }
     }
+  };
+  if (rows_here > 0) load(0, a[0]);
+  for (int r0 = 0; r0 < rows_here; r0 += 128) {
+    if (r0 + 64 < rows_here) load(r0 + 64, a[1]);
+    score(r0, a[0]);
+    if (r0 + 64 >= rows_here) break;
+    if (r0 + 128 < rows_here) load(r0 + 128, a[0]);
+    score(r0 + 64, a[1]);
   }
 }
 
