@@ -31,6 +31,9 @@
  *     by the caller; the library never allocates or frees, and keeps no state between calls.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and runs
  *     asynchronously; no entry point synchronises the host except lisa_check_device_error.
+ *   - The decode-path kernels are launched with programmatic dependent launch, so one may start
+ *     while the previous kernel of the stream drains; each waits for all earlier work of the stream
+ *     before it reads or writes memory that work may touch, so stream-order semantics are unchanged.
  *   - Arguments are checked on the host before anything is enqueued.  Any return other than LISA_OK
  *     from the checks means nothing was enqueued.  A failed launch returns LISA_ERR_CUDA.
  *   - Values that can only be checked on the device (sequence lengths, page ids, indices, counts) are
