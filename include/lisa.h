@@ -160,7 +160,9 @@ lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const 
  * of a KV head form the N side of one tensor-core contraction per 16-position tile (E4M3 -> f16 is
  * exact; each query as an f16 hi/lo pair, fp32 accumulation), so the scores agree with an fp32 dot
  * product to rounding.  Top-M per token: lisa_topm_select on a desc with B*T sequences (b*T + j,
- * length n_b - T + j + 1) over the same scores buffer. */
+ * length n_b - T + j + 1) over the same scores buffer.  Two kernels on `stream`: the first forms
+ * the T projected queries of each (b, KV head) into ws (the region the fused top-M keeps its
+ * candidates in), the second streams the projected keys once for all T tokens. */
 lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens, const void* q, const float* P,
                                    const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
                                    float* scores, void* ws, size_t ws_bytes, lisa_stream_t stream);

@@ -92,7 +92,9 @@ Layout layout_of(const lisa_decode_desc& d) {
   L.off_acount = off;
   off += align256(B * Hkv * 4);
   L.off_cand = off;
-  off += align256(B * Hkv * (size_t)L.cap * 8);
+  // The multi-query indexer keeps its projected queries here instead ([B][T][Hkv][32] fp32).
+  const size_t cand_bytes = (size_t)L.cap * 8 > (size_t)kMultiMaxT * 32 * 4 ? (size_t)L.cap * 8 : (size_t)kMultiMaxT * 32 * 4;
+  off += align256(B * Hkv * cand_bytes);
   L.total = off;
   return L;
 }
@@ -348,7 +350,7 @@ lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens,
   LISA_TRY(check_desc(desc));
   if (desc->batch == 0) return LISA_OK;
   LISA_TRY(check_idx_dim(desc));
-  if (num_tokens < 1 || num_tokens > 8) return LISA_ERR_UNSUPPORTED;
+  if (num_tokens < 1 || num_tokens > kMultiMaxT) return LISA_ERR_UNSUPPORTED;
   if (kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_UNSUPPORTED;
   if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || scores == nullptr)
     return LISA_ERR_INVALID_ARG;
@@ -375,6 +377,7 @@ lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens,
   p.kproj = kproj_pool;
   p.kproj_scale = kproj_scale;
   p.scores = scores;
+  p.uq = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.off_cand);
   p.err = static_cast<uint32_t*>(ws);
   return cuda_status(launch_index_score_multi(p, reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -22,6 +22,7 @@ constexpr int kAttnMaxTiles = 16;     // 64-position tiles per attention CTA, at
 constexpr int kMaxG = 8;              // query heads per KV head (mma n = 8)
 constexpr int kMaxSeqLen = 262144;
 constexpr int kMaxBudget = 16384;
+constexpr int kMultiMaxT = 8;        // query tokens per sequence of the multi-query indexer
 constexpr size_t kErrBytes = 256;     // head of the workspace: error word
 
 // Error word lives at the start of the workspace.
@@ -67,6 +68,25 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Four E4M3 values packed in a word -> two f16x2 words (bytes 0,1 -> lo; bytes 2,3 -> hi); exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 b0, b1;\n\t"
+      "mov.b32 {b0, b1}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, b0;\n\tcvt.rn.f16x2.e4m3x2 %1, b1;\n\t}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
+// D(16x8 fp32) += A(16x16 f16, row) * B(16x8 f16, col).
+__device__ __forceinline__ void mma_f16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,

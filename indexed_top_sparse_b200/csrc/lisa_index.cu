@@ -6,11 +6,11 @@
 // (a tie at the M-th score goes to the lower position) and reported in ascending order.
 //
 // Design on B200:
-//  * Scoring streams the projected-key cache; each lane owns whole rows (one 256-bit load per
-//    32-byte FP8 row, so a warp reads 1 KB of one page block at a time) and keeps up to eight rows
-//    in flight.  FP8 is decoded with the hardware e4m3x2 -> f16x2 conversion and accumulated with
-//    packed fp32x2 FMAs on the CUDA cores (a single query makes this a matrix-vector product: no
-//    tensor-core work to be had).
+//  * Scoring streams the projected-key cache: each warp moves its own range of rows through a
+//    private cp.async ring in shared memory.  FP8 rows are scored on the tensor cores as 16-row
+//    tiles (E4M3 -> f16 is exact, the projected query is split into f16 hi and lo parts, fp32
+//    accumulation), which takes the per-row convert-and-FMA chain off the issue slots; fp32 rows
+//    use packed fp32x2 FMAs on the CUDA cores.
 //  * The fused top-M never writes the fp32 scores to HBM: a sampled threshold lets the streaming
 //    kernel keep only ~2M candidates per (b, KV head) (see the sample / stream / finish kernels);
 //    the finish kernel does the exact selection on those, with an exact re-scoring fallback.
@@ -96,25 +96,6 @@ __device__ __forceinline__ float row_dot(const uint32_t* w, const float2* u2) {
     }
   }
   return (a0.x + a1.x) + (a0.y + a1.y);
-}
-
-// Four E4M3 values packed in a word -> two f16x2 words (bytes 0,1 -> lo; bytes 2,3 -> hi); exact.
-__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b16 b0, b1;\n\t"
-      "mov.b32 {b0, b1}, %2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, b0;\n\tcvt.rn.f16x2.e4m3x2 %1, b1;\n\t}\n"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
-
-// D(16x8 fp32) += A(16x16 f16, row) * B(16x8 f16, col).
-__device__ __forceinline__ void mma_f16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                              uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Projected-key scores of FP8 rows on the tensor cores.  The score is a dot product over the r
@@ -917,158 +898,6 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
   }
 }
 
-// Multi-query indexer scores (lisa_index_score_multi): T query tokens per sequence.  Token j of
-// sequence b sees positions t <= n_b - T + j; s[b][j][h][t] = scale_h <P_h qbar_{b,j,h}, c_t>.  The
-// T projected queries of a KV head are the columns of one tensor-core contraction over 16-row tiles
-// of FP8 projected keys: column pair (2j, 2j+1) holds u_j as 2^E_j (hi + lo) in f16, so lane (g, t)
-// of a warp finds query 4 nt + t of n-tile nt for rows g and g + 8 of every tile.  The A fragments
-// are loaded straight from the page blocks (8 consecutive rows of 32 bytes per lane group).
-constexpr int kMultiMaxT = 8;
-constexpr int kMultiChunk = 4096;
-constexpr int kMultiThreads = 128;
-
-template <int R>
-__global__ void __launch_bounds__(kMultiThreads) lisa_score_multi_kernel(MultiParams p) {
-  __shared__ float qbar[kMultiMaxT][128];
-  __shared__ float ush[kMultiMaxT][32];
-  __shared__ const uint8_t* pbase[kMultiChunk / 16];
-  constexpr int RB = R;                       // FP8: one byte per dimension
-  constexpr int NT = (2 * kMultiMaxT) / 8;    // n-tiles of 8 columns
-  constexpr int KS = R / 16;                  // k-steps of 16 dimensions
-  const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t4 = lane & 3;
-  const int T = p.T, G = p.Hq / p.Hkv, d = p.d;
-  int n = p.seq_lens[b];
-  if (n < 0 || n > p.max_seq_len) {
-    if (tid == 0) flag_error(p.err, LISA_DEVERR_SEQ_LEN);
-    n = n < 0 ? 0 : p.max_seq_len;
-  }
-  const int t_begin = blockIdx.x * kMultiChunk;
-  if (t_begin >= n) return;
-  const int nrows = min(n - t_begin, kMultiChunk);
-  // Projected queries of the T tokens (every CTA of the pair forms them; they are tiny).
-  for (int e = tid; e < T * d; e += blockDim.x) {
-    const int j = e / d, k = e % d;
-    float acc = 0.f;
-    for (int gg = 0; gg < G; ++gg) acc += __bfloat162float(p.q[(((size_t)b * T + j) * p.Hq + (size_t)h * G + gg) * d + k]);
-    qbar[j][k] = acc / (float)G;
-  }
-  {
-    const int npg = (nrows + p.ps - 1) >> p.log2ps;
-    for (int i = tid; i < npg; i += blockDim.x) {
-      int pid = p.page_table[(size_t)b * p.max_pages + (t_begin >> p.log2ps) + i];
-      if (pid < 0 || pid >= p.num_pages) {
-        flag_error(p.err, LISA_DEVERR_PAGE_ID);
-        pid = 0;
-      }
-      pbase[i] = reinterpret_cast<const uint8_t*>(p.kproj) + ((((size_t)pid * p.Hkv + h) << p.log2ps) * RB);
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < T * R; e += blockDim.x) {
-    const int j = e / R, i = e % R;
-    const float* Pr = p.P + ((size_t)h * R + i) * d;
-    float acc = 0.f;
-    for (int k = 0; k < d; ++k) acc = fmaf(Pr[k], qbar[j][k], acc);
-    ush[j][i] = acc;
-  }
-  __syncthreads();
-  // B fragments: lane (g, t4) holds column g of each n-tile, i.e. query (8 nt + g) / 2, part g & 1.
-  uint32_t bf[NT][KS][2];
-  float fac[NT];  // output scale of query 4 nt + t4
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int col = 8 * nt + g, j = col >> 1;
-    float mx = 0.f;
-    if (j < T)
-      for (int i = 0; i < R; ++i) mx = fmaxf(mx, fabsf(ush[j][i]));
-    const int E = mx > 0.f ? ilogbf(mx) - 13 : 0;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int e0 = (R / 4) * t4 + 4 * ks + 2 * jj;
-        __half v[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const float x = j < T ? ldexpf(ush[j][e0 + q], -E) : 0.f;
-          const __half hi = __float2half_rn(x);
-          v[q] = (col & 1) ? __float2half_rn(x - __half2float(hi)) : hi;
-        }
-        bf[nt][ks][jj] = (uint32_t)__half_as_ushort(v[0]) | ((uint32_t)__half_as_ushort(v[1]) << 16);
-      }
-    }
-    const int jo = 4 * nt + t4;  // the query whose score this lane receives from n-tile nt
-    float mo = 0.f;
-    if (jo < T)
-      for (int i = 0; i < R; ++i) mo = fmaxf(mo, fabsf(ush[jo][i]));
-    const int Eo = mo > 0.f ? ilogbf(mo) - 13 : 0;
-    fac[nt] = p.kproj_scale[h] * ldexpf(1.f, Eo);
-  }
-  // Each warp scores its quarter of the chunk, 16-row tiles, four tiles per batch of loads.
-  const int wrows = kMultiChunk / 4, w0 = warp * wrows;
-  const int rows_here = max(0, min(nrows - w0, wrows));
-  auto row_ptr = [&](int lr) { return pbase[lr >> p.log2ps] + (lr & (p.ps - 1)) * RB + (RB / 4) * t4; };
-  // Software pipeline: the next 64 rows' fragments are in flight while the current ones are used.
-  uint32_t a[2][4][2][R / 16];  // [buffer][tile][row g / g + 8][word]
-  auto load = [&](int r0, uint32_t (&buf)[4][2][R / 16]) {
-#pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int lr = w0 + r0 + 16 * tt + g + 8 * hh;
-        const bool ok = lr < w0 + rows_here;
-        const uint8_t* src = row_ptr(ok ? lr : w0);
-        if constexpr (R == 32) {  // read-only loads: free to move ahead of the score stores
-          const uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0u, 0u);
-          buf[tt][hh][0] = v.x;
-          buf[tt][hh][1] = v.y;
-        } else {
-          buf[tt][hh][0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(src)) : 0u;
-        }
-      }
-    }
-  };
-  float* __restrict__ out_scores = p.scores;
-  auto score = [&](int r0, const uint32_t (&buf)[4][2][R / 16]) {
-#pragma unroll
-    for (int tt = 0; tt < 4; ++tt) {
-      float dacc[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) dacc[nt][0] = dacc[nt][1] = dacc[nt][2] = dacc[nt][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        uint32_t a0, a1, a2, a3;
-        e4m3x4_to_f16x2(buf[tt][0][ks], a0, a2);
-        e4m3x4_to_f16x2(buf[tt][1][ks], a1, a3);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_f16_16816(dacc[nt], a0, a1, a2, a3, bf[nt][ks][0], bf[nt][ks][1]);
-      }
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int j = 4 * nt + t4;
-        if (j >= T) continue;
-        const int lim = n - T + j;  // last position token j sees
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int pos = t_begin + w0 + r0 + 16 * tt + g + 8 * hh;
-          if (pos <= lim && pos - t_begin < w0 + rows_here)
-            out_scores[(((size_t)b * T + j) * p.Hkv + h) * p.max_seq_len + pos] =
-                fac[nt] * (dacc[nt][2 * hh] + dacc[nt][2 * hh + 1]);
-        }
-      }
-    }
-  };
-  if (rows_here > 0) load(0, a[0]);
-  for (int r0 = 0; r0 < rows_here; r0 += 128) {
-    if (r0 + 64 < rows_here) load(r0 + 64, a[1]);
-    score(r0, a[0]);
-    if (r0 + 64 >= rows_here) break;
-    if (r0 + 128 < rows_here) load(r0 + 128, a[0]);
-    score(r0 + 64, a[1]);
-  }
-}
-
 }  // namespace
 
 size_t select_smem_bytes(int chunk_max, int ps) {
@@ -1377,15 +1206,6 @@ template <int R, bool FP8>
 static cudaError_t launch_score_t(const IndexParams& p, cudaStream_t stream) {
   dim3 grid((p.max_seq_len + kScoreChunk - 1) / kScoreChunk, p.Hkv, p.B);
   lisa_score_kernel<R, FP8><<<grid, kIndexThreads, 0, stream>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream) {
-  const dim3 grid((p.max_seq_len + kMultiChunk - 1) / kMultiChunk, p.Hkv, p.B);
-  if (p.r == 16)
-    lisa_score_multi_kernel<16><<<grid, kMultiThreads, 0, stream>>>(p);
-  else
-    lisa_score_multi_kernel<32><<<grid, kMultiThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -82,6 +82,7 @@ struct MultiParams {
   const void* kproj;       // FP8 E4M3 [num_pages][Hkv][ps][r]
   const float* kproj_scale;
   float* scores;           // [B][T][Hkv][max_seq_len]
+  float* uq;               // workspace: projected queries [B][T][Hkv][32]
   uint32_t* err;
 };
 

@@ -18,7 +18,8 @@ def _bits16(t):
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-@pytest.mark.parametrize("T,r,d,page", [(4, 32, 128, 64), (8, 32, 128, 16), (1, 16, 64, 64), (3, 16, 128, 1024)])
+@pytest.mark.parametrize("T,r,d,page", [(4, 32, 128, 64), (8, 32, 128, 16), (1, 16, 64, 64), (3, 16, 128, 1024),
+                                          (6, 32, 128, 256), (2, 16, 128, 32), (5, 16, 64, 128)])
 def test_multi_query_scores_and_selection(cuda_device, T, r, d, page):
     prob = make_problem(name="mq", device=cuda_device, B=2, Hq=8, Hkv=2, d=d, r=r, M=128,
                         seq_lens=[6000, 700], page_size=page, paged=True, kproj_fp8=True, plant=("cosine", 0.01),
