@@ -13,7 +13,6 @@ namespace {
 
 using namespace lisa;
 
-constexpr int kTargetAttnCtas = 148 * 2 * 4;  // SMs x resident CTAs x waves worth of partitions
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 inline bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }

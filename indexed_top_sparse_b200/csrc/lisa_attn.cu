@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   if (bad & LISA_DEVERR_PAGE_ID) flag_error(p.err, LISA_DEVERR_PAGE_ID);
   __syncthreads();
 
-  float m_run[2], l_run[2];  // per head 2t_, 2t_+1 (log2 units); l is a partial over this lane's rows
+  float m_run[2] = {kNegInf, kNegInf}, l_run[2] = {0.f, 0.f};  // per head 2t_, 2t_+1 (log2 units); l is a partial over this lane's rows
   float o[D / 16][4];
   uint32_t qf[D / 16][2];  // Q^T fragments (B operand, k = d, n = query head of the group)
   int cur = -1, cur_cnt = 0;

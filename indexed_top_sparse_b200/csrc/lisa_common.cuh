@@ -50,8 +50,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
 // start while the previous kernel of the stream still runs: pdl_wait() returns once that kernel
 // has completed and its writes are visible, and pdl_trigger() lets the next kernel start
-// launching.  The kernels here trigger only after their own wait, so a successor never starts
-// before all earlier work of the stream has completed.  Both are no-ops without the attribute.
+// launching.  The kernels here trigger only after their own wait, and every CTA waits before it
+// exits, even one with nothing to do: a grid then completes only after all earlier work of the
+// stream has, and a successor never starts before that.  Both are no-ops without the attribute.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 

@@ -719,55 +719,86 @@ constexpr int kStreamChunk = 4096;        // positions per streaming CTA
 constexpr int kStreamStageBytes = 2048;   // projected-key bytes per warp pipeline stage
 constexpr int kStreamStages = 4;          // stages in each warp's shared-memory ring
 constexpr int kStreamThreads = 128;       // threads of a streaming CTA (4 warps, 1024 positions each)
-constexpr int kStreamCtasPerSm = 5;       // resident streaming CTAs per SM (shared memory bound)
+constexpr int kStreamCtasPerSm = 6;       // resident streaming CTAs per SM (shared memory bound)
+constexpr int kWarpStage = 128;           // candidates a warp stages in shared memory between flushes
+
+// 32-bit load that stays where it is written (issued before the loads that follow it in source).
+__device__ __forceinline__ int ld_pinned_s32(const int32_t* ptr) {
+  int v;
+  asm volatile("ld.global.s32 %0, [%1];\n" : "=r"(v) : "l"(ptr));
+  return v;
+}
 
 // Each warp streams its own contiguous quarter of the CTA's chunk through a private cp.async ring:
-// a lane waits only for its own copies and the warp synchronises with __syncwarp, so the streaming
-// loop has no CTA-wide barrier.  Stage s of a warp holds rows [s * RPS, (s + 1) * RPS) of its range
-// (for fp32 rows, 16-byte chunks XOR-swizzled within each row so that the row reads are free of
-// bank conflicts).  Positions whose key reaches the threshold are staged in shared memory (one
-// shared atomic per lane that has any) and appended to the pair's candidate buffer at the end.
+// a lane waits only for its own copies and the warp synchronises with __syncwarp, so the kernel has
+// no CTA-wide barrier after its prologue.  Stage s of a warp holds rows [s * RPS, (s + 1) * RPS) of
+// its range (for fp32 rows, 16-byte chunks XOR-swizzled within each row so that the row reads are
+// free of bank conflicts).  The page ids of a warp's range live in its lanes' registers and are
+// fetched together with the sequence length.  Positions whose key reaches the threshold are staged
+// per warp in shared memory (slots from a warp prefix sum) and appended to the pair's candidate
+// buffer, one global atomic per flush, whenever the stage would overflow and at the end.
 template <int R, bool FP8>
 __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_stream_kernel(IndexParams p) {
   extern __shared__ __align__(128) uint8_t ring[];  // [warp][kStreamStages][kStreamStageBytes]
-  __shared__ const uint8_t* pbase[kStreamChunk / 16];  // global address of each page block of the chunk
-  __shared__ uint32_t ckey[kStageCap];
-  __shared__ uint32_t cpos[kStageCap];
-  __shared__ uint32_t s_ncand, s_base;
+  constexpr int WARPS = kStreamThreads / 32;
+  __shared__ uint2 cstage[WARPS][kWarpStage];      // (key, position) staged by each warp
   using Geo = RowGeom<R, FP8>;
   constexpr int RB = Geo::kRowBytes;
   constexpr int CPR = RB / 16;                            // 16-byte chunks per row
   constexpr int RPS = kStreamStageBytes / RB;             // rows per stage
   constexpr int RPL = RPS >= 32 ? RPS / 32 : 1;           // rows per lane per stage
-  constexpr int WARPS = kStreamThreads / 32;
   constexpr int WROWS = kStreamChunk / WARPS;             // rows per warp
+  constexpr int kPidRegs = (WROWS / 16 + 31) / 32;        // page ids per lane at the smallest page size
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * p.Hkv + h;
-  const int n = load_seq_len(p, b);
-  if (n <= p.M) return;
   const int t_begin = blockIdx.x * kStreamChunk;
-  if (t_begin >= n) return;
+  const int w0 = warp * WROWS;  // first row of this warp (chunk-relative)
+  // The warp's range lies in max(1, WROWS / ps) whole page blocks (both are powers of two, and the
+  // range starts on a multiple of WROWS): lane l holds the id of block l + 32 k of it.  The ids are
+  // inputs of the step, loaded before the wait and together with the sequence length.
+  const int pg0 = (t_begin + w0) >> p.log2ps;
+  const int npw = WROWS > p.ps ? (WROWS >> p.log2ps) : 1;
+  int pid[kPidRegs];
+#pragma unroll
+  for (int k = 0; k < kPidRegs; ++k) {
+    const int rel = lane + 32 * k;
+    pid[k] = (rel < npw && pg0 + rel < p.max_pages) ? ld_pinned_s32(p.page_table + (size_t)b * p.max_pages + pg0 + rel) : 0;
+  }
+  const int n = load_seq_len(p, b);
+  if (n <= p.M || t_begin >= n) {
+    pdl_wait();  // no CTA ends before the earlier kernels of the stream have completed
+    return;
+  }
   const int nrows = min(n - t_begin, kStreamChunk);
-  if (tid == 0) s_ncand = 0u;
-  {
-    const int npg = (nrows + p.ps - 1) >> p.log2ps;
-    const uint8_t* base = reinterpret_cast<const uint8_t*>(p.kproj);
-    for (int i = tid; i < npg; i += blockDim.x) {
-      int pid = p.page_table[(size_t)b * p.max_pages + (t_begin >> p.log2ps) + i];
-      if (pid < 0 || pid >= p.num_pages) {
-        flag_error(p.err, LISA_DEVERR_PAGE_ID);
-        pid = 0;
-      }
-      pbase[i] = base + ((((size_t)pid * p.Hkv + h) << p.log2ps) * RB);
+  const int wrows = max(0, min(nrows - w0, WROWS));  // rows this warp scores
+  const int nstages = (wrows + RPS - 1) / RPS;
+#pragma unroll
+  for (int k = 0; k < kPidRegs; ++k) {
+    const int rel = lane + 32 * k;
+    const bool used = rel < npw && (long long)rel * p.ps < wrows;
+    if (!used) {
+      pid[k] = 0;
+    } else if (pid[k] < 0 || pid[k] >= p.num_pages) {
+      flag_error(p.err, LISA_DEVERR_PAGE_ID);
+      pid[k] = 0;
     }
   }
-  __syncthreads();
+  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(p.kproj);
+  // Address of warp-relative row r (r < wrows); every lane of the warp calls it together.
+  auto row_src = [&](int r) -> const uint8_t* {
+    const int t = t_begin + w0 + r;
+    const int rel = (t >> p.log2ps) - pg0;
+    int id = __shfl_sync(0xffffffffu, pid[0], rel & 31);
+#pragma unroll
+    for (int k = 1; k < kPidRegs; ++k) {
+      const int idk = __shfl_sync(0xffffffffu, pid[k], rel & 31);
+      if ((rel >> 5) == k) id = idk;
+    }
+    return kbase + ((((size_t)id * p.Hkv + h) << p.log2ps) + (t & (p.ps - 1))) * RB;
+  };
 
   uint8_t* wring = ring + warp * (kStreamStages * kStreamStageBytes);
-  const int w0 = warp * WROWS;                               // first row of this warp (chunk-relative)
-  const int wrows = max(0, min(nrows - w0, WROWS));          // rows this warp scores
-  const int nstages = (wrows + RPS - 1) / RPS;
   // FP8 rows are read as 16-row tensor-core tiles (8 consecutive rows per lane group: no bank
   // conflicts unswizzled); fp32 rows are read one per lane, with 16-byte chunks XOR-swizzled.
   auto swz_off = [&](int r, int part) {
@@ -778,8 +809,7 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
     uint8_t* dst = wring + (stage % kStreamStages) * kStreamStageBytes;
     if (FP8 && p.ps >= RPS) {
       // the stage's rows are contiguous inside one page block: one base, unswizzled 16-byte chunks
-      const int lr0 = w0 + stage * RPS;
-      const uint8_t* base = pbase[lr0 >> p.log2ps] + (lr0 & (p.ps - 1)) * RB;
+      const uint8_t* base = row_src(stage * RPS);
       const int vbytes = min(RPS, wrows - stage * RPS) * RB;
 #pragma unroll
       for (int k = 0; k < kStreamStageBytes / 512; ++k) {
@@ -792,10 +822,9 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
     for (int k = 0; k < kStreamStageBytes / 512; ++k) {
       const int c = lane + 32 * k;  // 16-byte chunk of the stage
       const int r = c / CPR, part = c % CPR;
-      const int lr = w0 + stage * RPS + r;
-      const bool valid = r < RPS && lr < w0 + wrows;
-      const int vr = valid ? lr : w0;
-      const uint8_t* src = pbase[vr >> p.log2ps] + (vr & (p.ps - 1)) * RB + part * 16;
+      const int lr = stage * RPS + r;  // warp-relative row
+      const bool valid = r < RPS && lr < wrows;
+      const uint8_t* src = row_src(valid ? lr : 0) + part * 16;
       cp_async_16(smem_u32(dst + swz_off(r, part)), src, valid ? 16u : 0u);
     }
   };
@@ -817,6 +846,22 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
     mma_score.init(p.uq + bh * 32, scale, lane);
   else
     load_u2<R>(p.uq + bh * 32, u2);
+  // Appends the warp's staged candidates to the pair's buffer (one global atomic); entries past
+  // the capacity are dropped, and the count then tells the finish step to take the exact path.
+  uint32_t wn = 0u;  // candidates staged by this warp (the same in every lane)
+  uint2* cdst = reinterpret_cast<uint2*>(p.cand) + bh * (size_t)p.cap;
+  auto flush = [&]() {
+    __syncwarp();
+    if (wn == 0u) return;
+    uint32_t base = 0u;
+    if (lane == 0) base = atomicAdd(&p.ccount[bh], wn);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    for (uint32_t i = lane; i < wn; i += 32u) {
+      const uint32_t slot = base + i;
+      if (slot < (uint32_t)p.cap) cdst[slot] = cstage[warp][i];
+    }
+    __syncwarp();
+  };
   for (int st = 0; st < nstages; ++st) {
     issue(st + kStreamStages - 1);
     cp_async_commit();
@@ -869,33 +914,34 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
         if (r < RPS && st * RPS + r < wrows && key[k] >= tau) mask |= 1u << k;
       }
     }
-    if (mask != 0u) {  // a few lanes per stage: one shared-memory atomic each
-      uint32_t slot = atomicAdd(&s_ncand, (uint32_t)__popc(mask));
+    // Stage this stage's candidates: slots from a warp prefix sum of the per-lane counts.
+    if (__any_sync(0xffffffffu, mask != 0u)) {
+      const uint32_t c = (uint32_t)__popc(mask);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+      if (wn + tot > (uint32_t)kWarpStage) {
+        flush();
+        wn = 0u;
+      }
+      uint32_t slot = wn + incl - c;
 #pragma unroll
       for (int k = 0; k < NK; ++k) {
         if ((mask >> k) & 1u) {
-          if (slot < (uint32_t)kStageCap) {
-            ckey[slot] = key[k];
-            cpos[slot] = (uint32_t)(t_begin + w0 + st * RPS + rloc[k]);
-          }
+          cstage[warp][slot] = make_uint2(key[k], (uint32_t)(t_begin + w0 + st * RPS + rloc[k]));
           ++slot;
         }
       }
+      wn += tot;
     }
-    __syncwarp();  // the slot is refilled by a later stage
+    __syncwarp();  // the ring slot is refilled by a later stage
   }
   cp_async_wait<0>();
-  __syncthreads();
-  const uint32_t nc = s_ncand;
-  if (nc == 0u) return;
-  if (tid == 0) s_base = atomicAdd(&p.ccount[bh], nc <= (uint32_t)kStageCap ? nc : (uint32_t)p.cap + 1u);
-  __syncthreads();
-  if (nc > (uint32_t)kStageCap) return;  // the count now exceeds the capacity: the exact path runs
-  uint2* dst = reinterpret_cast<uint2*>(p.cand) + bh * (size_t)p.cap;
-  for (uint32_t i = tid; i < nc; i += blockDim.x) {
-    const uint32_t slot = s_base + i;
-    if (slot < (uint32_t)p.cap) dst[slot] = make_uint2(ckey[i], cpos[i]);
-  }
+  flush();
 }
 
 }  // namespace
@@ -1147,9 +1193,9 @@ __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(Index
   extern __shared__ __align__(16) uint32_t fsm[];
   const int h = blockIdx.x, b = blockIdx.y;
   const int n = load_seq_len(p, b);
-  if (n <= p.M) return;  // the sample kernel wrote the full set
   pdl_wait();  // candidates and counts come from the streaming kernel
   pdl_trigger();
+  if (n <= p.M) return;  // the sample kernel wrote the full set
   uint32_t* cstage = fsm + 2 * finish_bitmap_words(p.max_seq_len);
   finish_pair<R, FP8, kFinishThreads>(p, b, h, n, fsm, cstage, finish_stage_cap(p.cap));
 }
@@ -1184,6 +1230,7 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
   const size_t ring = (size_t)(kStreamThreads / 32) * kStreamStages * kStreamStageBytes;
   auto k = lisa_index_stream_kernel<R, FP8>;
   e = set_smem(k, ring);
+  if (e == cudaSuccess) e = prefer_max_smem(k);
   if (e != cudaSuccess) return e;
   e = launch_pdl(k, grid, dim3(kStreamThreads), ring, stream, p);
   if (e != cudaSuccess) return e;

@@ -10,7 +10,6 @@ namespace lisa {
 
 constexpr int kScoreChunk = 4096;   // positions per CTA of the score-only and streaming kernels
 constexpr int kSampleMax = 4096;    // positions the threshold sample scores per (b, KV head)
-constexpr int kStageCap = 1024;     // candidates a streaming CTA can stage in shared memory
 
 struct IndexParams {
   int B, Hq, Hkv, d, r, M, ps, log2ps, max_pages, max_seq_len, num_pages;
@@ -139,6 +138,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Shared-memory-bound streaming kernels ask for the largest shared memory carve-out, so that their
+// occupancy is set by shared memory alone (they read global memory through L2 only).
+template <typename... KArgs>
+inline cudaError_t prefer_max_smem(void (*kernel)(KArgs...)) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
 }
 
 // after_sample / after_stream: optional events recorded between the three kernels (nullptr: none).

@@ -29,7 +29,7 @@ constexpr int kMultiChunk = 4096;       // positions per scoring CTA
 constexpr int kMultiThreads = 128;      // 4 warps, 1024 positions each
 constexpr int kMultiStageBytes = 2048;  // projected-key bytes per warp pipeline stage
 constexpr int kMultiStages = 4;         // stages in each warp's shared-memory ring
-constexpr int kMultiCtasPerSm = 5;
+constexpr int kMultiCtasPerSm = 6;
 
 // uq[b][j][h][0..r): the projected mean query of token j (fp32, 32 slots per row).
 __global__ void __launch_bounds__(kMultiThreads) lisa_multi_project_kernel(MultiParams p) {
@@ -256,6 +256,8 @@ template <int R, int NT>
 cudaError_t launch_score_multi_t(const MultiParams& p, cudaStream_t stream) {
   const size_t smem = (size_t)(kMultiThreads / 32) * kMultiStages * kMultiStageBytes;
   const dim3 grid((p.max_seq_len + kMultiChunk - 1) / kMultiChunk, p.Hkv, p.B);
+  cudaError_t e = prefer_max_smem(lisa_score_multi_kernel<R, NT>);
+  if (e != cudaSuccess) return e;
   return launch_pdl(lisa_score_multi_kernel<R, NT>, grid, dim3(kMultiThreads), smem, stream, p);
 }
 
