@@ -410,3 +410,35 @@ def test_fused_topm_too_few_candidates_falls_back_exactly(cuda_device):
     assert len(same) == len(all_pairs(prob))
     for h in range(prob.Hkv):
         assert set(hot.tolist()) <= set(idx[0, h].tolist())
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_fused_topm_concentrated_candidates(cuda_device, fp8):
+    # A contiguous block of high scores: most candidates land in one warp's range of one streaming
+    # chunk, so that warp's shared-memory stage is flushed to the candidate buffer many times over.
+    n, M = 20000, 1024
+    prob = small(cuda_device, B=1, Hq=8, Hkv=2, d=128, r=32, M=M, seq_lens=[n], paged=True, kproj_fp8=fp8,
+                 plant=("none",), seed=97)
+    blk = torch.arange(4096, 4096 + 1500)
+    g = torch.Generator().manual_seed(5)
+    G = prob.G
+    for h in range(prob.Hkv):
+        qbar = prob.q[0, h * G : (h + 1) * G].double().mean(0)
+        u = prob.P[h].double().cpu() @ qbar.cpu()
+        alpha = 0.5 + 0.5 * torch.rand(len(blk), 1, generator=g, dtype=torch.float64)
+        rows = (alpha * 440.0 * u / u.abs().max()).float()
+        if fp8:
+            rows = rows.to(torch.float8_e4m3fn).view(torch.uint8)
+        pages = prob.page_table[0, blk // prob.page_size].long().to(cuda_device)
+        prob.kproj[pages, h, (blk % prob.page_size).to(cuda_device)] = rows.to(cuda_device)
+    ws = R.workspace(prob)
+    idx, count = R.index_topm(prob, ws)
+    assert L.lisa_check_device_error(ws) == 0
+    inp = host_inputs(prob)
+    ref = O.decode_step(inp)
+    same = check_index_sets(idx.cpu().numpy(), count.cpu().numpy(), ref, inp["seq_lens"], M, all_pairs(prob))
+    assert len(same) == len(all_pairs(prob))
+    for h in range(prob.Hkv):
+        assert int(count[0, h]) == M
+        # the input does what it is meant to: most of the top-M sits inside the block
+        assert len(set(ref["idx"][0][h].tolist()) & set(blk.tolist())) >= 900
