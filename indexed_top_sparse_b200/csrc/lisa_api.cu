@@ -23,7 +23,7 @@ inline int ilog2(int x) {
 }
 
 struct Layout {
-  int G = 0, grid = 0, tpp = 0, splits = 0, chunk_max = 0, cap = 0;  // splits: partial slots per pair
+  int G = 0, grid = 0, tpp = 0, splits = 0, cap = 0;  // splits: partial slots per pair
   size_t off_idx = 0, off_count = 0, off_opart = 0, off_ml = 0;
   size_t off_uq = 0, off_tau = 0, off_ccount = 0, off_acount = 0, off_cand = 0, total = 0;
 };
@@ -67,8 +67,6 @@ Layout layout_of(const lisa_decode_desc& d) {
   if (grid * kAttnMaxTiles < tiles) grid = (tiles + kAttnMaxTiles - 1) / kAttnMaxTiles;
   L.grid = (int)grid;
   L.splits = (int)((L.grid + pairs - 1) / pairs) + 1;
-  const int per_cta = (d.max_seq_len + kClusterSize - 1) / kClusterSize;
-  L.chunk_max = ((per_cta + d.page_size - 1) / d.page_size) * d.page_size;
   const size_t B = (size_t)d.batch, Hkv = (size_t)d.num_kv_heads;
   size_t off = kErrBytes;
   L.off_idx = off;
@@ -171,7 +169,6 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   p.max_pages = d.max_pages_per_seq;
   p.max_seq_len = d.max_seq_len;
   p.num_pages = d.num_pages;
-  p.chunk_max = L.chunk_max;
   p.cap = L.cap;
   p.seq_lens = d.seq_lens;
   p.page_table = d.page_table;
@@ -393,7 +390,7 @@ lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, 
   p.scores = const_cast<float*>(scores);
   p.idx = idx;
   p.count = count;
-  return cuda_status(launch_index_select(p, true, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_index_select(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_index_topm(const lisa_decode_desc* desc, const void* q, const float* P, const void* kproj_pool,

@@ -11,7 +11,6 @@
 
 namespace lisa {
 
-constexpr int kClusterSize = 8;       // CTAs cooperating on one (b, KV head) index set
 constexpr int kIndexThreads = 256;    // threads of an index-stage CTA
 constexpr int kBins = 2048;           // radix digits per pass (11 bits)
 constexpr int kAttnThreads = 128;     // threads of an attention CTA (4 warps)

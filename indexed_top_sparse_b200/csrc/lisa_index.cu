@@ -14,23 +14,18 @@
 //  * The fused top-M never writes the fp32 scores to HBM: a sampled threshold lets the streaming
 //    kernel keep only ~2M candidates per (b, KV head) (see the sample / stream / finish kernels);
 //    the finish kernel does the exact selection on those, with an exact re-scoring fallback.
-//  * Selection from caller-given scores uses a cluster of 8 CTAs per (b, KV head) with the
-//    histograms reduced over distributed shared memory.
-
-#include <cooperative_groups.h>
+//  * Selection from caller-given scores runs the same threshold pipeline on them: a sampled
+//    threshold, a filter kernel that streams the scores and keeps the keys above it, and the same
+//    exact finish (whose fallback then reads the scores instead of re-scoring).
 
 #include "lisa_common.cuh"
 #include "lisa_kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace lisa {
 
 namespace {
 
 
-constexpr int kCandCap = 2048;  // keys inside the threshold digit kept in a list, per CTA
-constexpr int kTieCap = 64;     // ties at the M-th key resolved from a list, per CTA
 
 template <int R, bool FP8>
 struct RowGeom {
@@ -243,38 +238,6 @@ __device__ __forceinline__ void stream_scores(const IndexParams& p, int h, int t
   }
 }
 
-struct SelectSmem {
-  uint32_t hist0[kBins];      // top 11 key bits
-  uint32_t hist1[kBins];      // next 11 bits, keys inside the pass-0 digit
-  uint32_t hist2[kBins / 2];  // last 10 bits
-  uint32_t cand_key[kCandCap];
-  uint32_t cand_pos[kCandCap];
-  uint32_t tie_pos[kTieCap];
-  uint32_t scan[32];
-  uint32_t digit[2];
-  uint32_t cnt[2];  // (#keys > K, #keys == K) of this CTA, read by the other CTAs of the cluster
-  uint32_t ncand, nabove, ngt, ntie;
-};
-
-// Sum of the cluster's histograms over this thread's PER consecutive bins, into registers.
-template <int PER>
-__device__ __forceinline__ void cluster_bins(cg::cluster_group& cluster, uint32_t* hist, uint32_t (&v)[PER]) {
-#pragma unroll
-  for (int i = 0; i < PER; ++i) v[i] = 0u;
-#pragma unroll
-  for (int r = 0; r < kClusterSize; ++r) {
-    const uint4* rh = reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, r) + threadIdx.x * PER);
-#pragma unroll
-    for (int q = 0; q < PER / 4; ++q) {
-      const uint4 a = rh[q];
-      v[4 * q + 0] += a.x;
-      v[4 * q + 1] += a.y;
-      v[4 * q + 2] += a.z;
-      v[4 * q + 3] += a.w;
-    }
-  }
-}
-
 // Block-wide: the bins (PER per thread, thread t owns bins [t*PER, (t+1)*PER), higher bin = larger
 // key) hold candidate counts; find the bin holding the need-th largest candidate.  Writes the bin
 // and the rank of that key inside it (1-based) to digit[0..1].  Ends with a barrier.
@@ -385,6 +348,33 @@ template <int R>
 __device__ __forceinline__ void load_u2(const float* u, float2* u2) {
 #pragma unroll
   for (int k = 0; k < R / 2; ++k) u2[k] = make_float2(u[2 * k], u[2 * k + 1]);
+}
+
+// Threshold key of the candidate filter: the lower edge of the 22-bit key bin that holds the
+// rank-th largest of the S sampled keys, rank = ceil(2 M S / n) + 16 (capped at S), i.e. about twice
+// the M-th largest's expected rank.  skey holds the sample keys and hist their top-11-bit histogram;
+// hist is reused.  Ends with a barrier; every thread returns the threshold.
+template <int THREADS>
+__device__ uint32_t sample_threshold(uint32_t* hist, const uint32_t* skey, int S, int n, int M, uint32_t* scan,
+                                     uint32_t* digit) {
+  const int tid = threadIdx.x;
+  const uint32_t rank = (uint32_t)min((long long)S, (2LL * M * S + n - 1) / n + 16);
+  constexpr int PER = kBins / THREADS;
+  uint32_t v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, rank, scan, digit);
+  const uint32_t d0 = digit[0], need = digit[1];
+  __syncthreads();
+  for (int i = tid; i < kBins; i += THREADS) hist[i] = 0u;
+  __syncthreads();
+  for (int j = tid; j < S; j += THREADS)
+    if ((skey[j] >> 21) == d0) atomicAdd(&hist[(skey[j] >> 10) & 0x7ffu], 1u);
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
+  find_digit(v, need, scan, digit);
+  return (d0 << 21) | (digit[0] << 10);
 }
 
 constexpr int kSampleThreads = 512;
@@ -519,30 +509,14 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   }
   if (bad) flag_error(p.err, bad);
   __syncthreads();
-  // tau: lower edge of the 22-bit key bin that holds the rank-th largest sample key
-  const uint32_t rank = (uint32_t)min((long long)S, (2LL * p.M * S + n - 1) / n + 16);
-  constexpr int PER = kBins / kSampleThreads;
-  uint32_t v[PER];
-#pragma unroll
-  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
-  find_digit(v, rank, scan, digit);
-  const uint32_t d0 = digit[0], need = digit[1];
-  __syncthreads();
-  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
-  __syncthreads();
-  for (int j = tid; j < S; j += blockDim.x)
-    if ((skey[j] >> 21) == d0) atomicAdd(&hist[(skey[j] >> 10) & 0x7ffu], 1u);
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < PER; ++i) v[i] = hist[tid * PER + i];
-  find_digit(v, need, scan, digit);
-  if (tid == 0) p.tau[bh] = (d0 << 21) | (digit[0] << 10);
+  const uint32_t tau = sample_threshold<kSampleThreads>(hist, skey, S, n, p.M, scan, digit);
+  if (tid == 0) p.tau[bh] = tau;
 }
 
 // Exact top-M of (b, h) (n > M) by the whole CTA, from the candidate buffer -- or, when it holds
 // fewer than M candidates or overflowed, by re-scoring every position.  fsm: two bitmaps of
 // ceil(n / 32) words, then room for `stage_cap` candidates staged from global memory.
-template <int R, bool FP8, int THREADS>
+template <int R, bool FP8, int THREADS, bool FROM_SCORES>
 __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t* fsm, uint32_t* cstage,
                             uint32_t stage_cap) {
   __shared__ uint32_t hist[kBins];
@@ -562,8 +536,11 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
   const bool fast = cnt >= (uint32_t)p.M && cnt <= (uint32_t)p.cap;
   const uint2* cand = reinterpret_cast<const uint2*>(p.cand) + bh * (size_t)p.cap;
   float2 u2[R / 2];
-  load_u2<R>(p.uq + bh * 32, u2);
-  const float scale = p.kproj_scale[h];
+  float scale = 0.f;
+  if constexpr (!FROM_SCORES) {
+    load_u2<R>(p.uq + bh * 32, u2);
+    scale = p.kproj_scale[h];
+  }
   // Candidates that fit are staged in shared memory once; the passes below then read them there.
   const bool staged = fast && cnt <= stage_cap;
   if (staged) {
@@ -608,6 +585,9 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
         const uint2 e = __ldcg(&cand[cnt - 1]);
         fn(e.x, e.y);
       }
+    } else if constexpr (FROM_SCORES) {
+      const float* sc = p.scores + bh * (size_t)p.max_seq_len;
+      for (int t = tid; t < n; t += blockDim.x) fn(score_key(__ldg(sc + t)), (uint32_t)t);
     } else {
       for (int t = tid; t < n; t += blockDim.x) {
         uint32_t w[RowGeom<R, FP8>::kWords];
@@ -944,251 +924,148 @@ __global__ void __launch_bounds__(kStreamThreads, kStreamCtasPerSm) lisa_index_s
   flush();
 }
 
-}  // namespace
 
-size_t select_smem_bytes(int chunk_max, int ps) {
-  (void)ps;
-  return sizeof(SelectSmem) + (size_t)chunk_max * 4 + (size_t)((chunk_max + 31) / 32) * 4;
-}
+// ---------------------------------------------------------------------------------------------
+// Top-M from caller-given fp32 scores (lisa_topm_select): the threshold pipeline of the fused
+// path, with the scores read instead of computed.
+// ---------------------------------------------------------------------------------------------
 
-// Top-M from caller-given fp32 scores (lisa_topm_select): one cluster of kClusterSize CTAs per
-// (b, KV head).  Each CTA loads a contiguous, page-aligned eighth of the scores into shared memory
-// as order-preserving uint32 keys with a histogram of the top 11 key bits; the histograms are
-// summed through distributed shared memory, one pass over the keys writes a bitmap of the keys
-// above the threshold digit and a list of the keys inside it, two more histogram passes pin the
-// exact M-th key, and each CTA emits its selected positions in ascending order.
-__global__ void __cluster_dims__(kClusterSize, 1, 1) __launch_bounds__(kIndexThreads, 2)
-    lisa_select_from_scores_kernel(IndexParams p) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectSmem));
-  uint32_t* bitmap = keys + p.chunk_max;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-  const uint32_t lt_mask = (1u << lane) - 1u;
+// Per (b, KV head): the sampled threshold key from the scores at the sample positions; the full
+// set when n <= M.
+__global__ void __launch_bounds__(kSampleThreads) lisa_select_sample_kernel(IndexParams p) {
+  __shared__ uint32_t hist[kBins];
+  __shared__ uint32_t skey[kSampleMax];
+  __shared__ uint32_t scan[32];
+  __shared__ uint32_t digit[2];
+  constexpr int SPT = kSampleMax / kSampleThreads;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  pdl_wait();  // first kernel of the call: the scores may come from earlier stream work
+  pdl_trigger();
   const int n = load_seq_len(p, b);
-  int32_t* idx_out = p.idx + ((size_t)b * p.Hkv + h) * p.M;
-
-  if (n <= p.M) {  // every position is kept; the whole cluster takes this branch together
-    for (int i = rank * blockDim.x + tid; i < p.M; i += kClusterSize * blockDim.x) idx_out[i] = i < n ? i : -1;
-    if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = n;
+  if (tid == 0) p.ccount[bh] = 0u;
+  if (n <= p.M) {  // every position is kept; the filter and finish kernels skip this pair
+    int32_t* idx_out = p.idx + bh * p.M;
+    for (int i = tid; i < p.M; i += blockDim.x) idx_out[i] = i < n ? i : -1;
+    if (tid == 0) {
+      p.tau[bh] = 0u;
+      p.count[bh] = n;
+    }
     return;
   }
-
-  // This CTA's page-aligned slice of the context.
-  const int chunk = ((((n + kClusterSize - 1) / kClusterSize) + p.ps - 1) >> p.log2ps) << p.log2ps;
-  const int t_begin = rank * chunk;
-  const int nrows = max(0, min(n, t_begin + chunk) - t_begin);
-  const int nwords = (nrows + 31) >> 5;
-
-  for (int i = tid; i < kBins; i += blockDim.x) {
-    sm.hist0[i] = 0u;
-    sm.hist1[i] = 0u;
-    if (i < kBins / 2) sm.hist2[i] = 0u;
+  const int S = min(n, kSampleMax);
+  const float* sc = p.scores + bh * (size_t)p.max_seq_len;
+  float v[SPT];
+#pragma unroll
+  for (int k = 0; k < SPT; ++k) {
+    const int j = tid + k * kSampleThreads;
+    v[k] = j < S ? __ldg(sc + sample_pos(j, n)) : 0.f;
   }
-  if (tid == 0) sm.ncand = sm.nabove = sm.ngt = sm.ntie = 0u;
+  for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
   __syncthreads();
-  const float* src = p.scores + ((size_t)b * p.Hkv + h) * p.max_seq_len + t_begin;
-  for (int lr = tid; lr < nrows; lr += blockDim.x) {
-    const uint32_t k = score_key(src[lr]);
-    keys[lr] = k;
-    atomicAdd(&sm.hist0[k >> 21], 1u);
-  }
-
-  // ---- pass 0: digit of the top 11 key bits holding the M-th key of (b, h)
-  cluster.sync();
-  {
-    uint32_t v[kBins / kIndexThreads];
-    cluster_bins(cluster, sm.hist0, v);
-    find_digit(v, (uint32_t)p.M, sm.scan, sm.digit);
-  }
-  const uint32_t d0 = sm.digit[0];
-  uint32_t need = sm.digit[1];
-
-  // One pass over the keys: bitmap words of keys above d0, list of keys inside d0.
-  const int wpw = (nwords + nwarps - 1) / nwarps;
-  {
-    uint32_t above = 0;
-    const int wb = warp * wpw, we = min(nwords, wb + wpw);
-    for (int word = wb; word < we; ++word) {
-      const int lr = word * 32 + lane;
-      const bool valid = lr < nrows;
-      const uint32_t k = valid ? keys[lr] : 0u;
-      const uint32_t dig = k >> 21;
-      const uint32_t bal = __ballot_sync(0xffffffffu, valid && dig > d0);
-      if (lane == 0) bitmap[word] = bal;
-      above += __popc(bal);
-      const bool cand = valid && dig == d0;
-      const uint32_t bc = __ballot_sync(0xffffffffu, cand);
-      if (bc) {
-        uint32_t base = 0;
-        if (lane == 0) base = atomicAdd(&sm.ncand, (uint32_t)__popc(bc));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (cand) {
-          const uint32_t slot = base + __popc(bc & lt_mask);
-          if (slot < (uint32_t)kCandCap) {
-            sm.cand_key[slot] = k;
-            sm.cand_pos[slot] = (uint32_t)lr;
-          }
-        }
-      }
-    }
-    if (lane == 0 && above) atomicAdd(&sm.nabove, above);
-  }
-  __syncthreads();
-  const uint32_t ncand = sm.ncand;
-  const bool listed = ncand <= (uint32_t)kCandCap;
-
-  // ---- pass 1: next 11 bits among keys inside d0
-  if (listed) {
-    for (uint32_t i = tid; i < ncand; i += blockDim.x) atomicAdd(&sm.hist1[(sm.cand_key[i] >> 10) & 0x7ffu], 1u);
-  } else {
-    for (int lr = tid; lr < nrows; lr += blockDim.x) {
-      const uint32_t k = keys[lr];
-      if ((k >> 21) == d0) atomicAdd(&sm.hist1[(k >> 10) & 0x7ffu], 1u);
-    }
-  }
-  cluster.sync();
-  {
-    uint32_t v[kBins / kIndexThreads];
-    cluster_bins(cluster, sm.hist1, v);
-    find_digit(v, need, sm.scan, sm.digit);
-  }
-  const uint32_t prefix22 = (d0 << 11) | sm.digit[0];
-  need = sm.digit[1];
-
-  // ---- pass 2: last 10 bits
-  if (listed) {
-    for (uint32_t i = tid; i < ncand; i += blockDim.x) {
-      const uint32_t k = sm.cand_key[i];
-      if ((k >> 10) == prefix22) atomicAdd(&sm.hist2[k & 0x3ffu], 1u);
-    }
-  } else {
-    for (int lr = tid; lr < nrows; lr += blockDim.x) {
-      const uint32_t k = keys[lr];
-      if ((k >> 10) == prefix22) atomicAdd(&sm.hist2[k & 0x3ffu], 1u);
-    }
-  }
-  cluster.sync();
-  {
-    uint32_t v[kBins / 2 / kIndexThreads];
-    cluster_bins(cluster, sm.hist2, v);
-    find_digit(v, need, sm.scan, sm.digit);
-  }
-  const uint32_t K = (prefix22 << 10) | sm.digit[0];  // the M-th largest key of (b, h)
-  const uint32_t tie_take = sm.digit[1];               // keys equal to K to keep, lowest positions first
-
-  // Keys inside d0 that are above K join the bitmap; keys equal to K are counted.
-  {
-    uint32_t gt = 0;
-    auto visit = [&](uint32_t k, uint32_t pos) {
-      if (k > K) {
-        atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
-        ++gt;
-      } else if (k == K) {
-        const uint32_t slot = atomicAdd(&sm.ntie, 1u);
-        if (slot < (uint32_t)kTieCap) sm.tie_pos[slot] = pos;
-      }
-    };
-    if (listed) {
-      for (uint32_t i = tid; i < ncand; i += blockDim.x) visit(sm.cand_key[i], sm.cand_pos[i]);
-    } else {
-      for (int lr = tid; lr < nrows; lr += blockDim.x) {
-        const uint32_t k = keys[lr];
-        if ((k >> 21) == d0) visit(k, (uint32_t)lr);
-      }
-    }
-    gt = __reduce_add_sync(0xffffffffu, gt);
-    if (lane == 0 && gt) atomicAdd(&sm.ngt, gt);
-  }
-  __syncthreads();
-  if (tid == 0) {
-    sm.cnt[0] = sm.nabove + sm.ngt;
-    sm.cnt[1] = sm.ntie;
-  }
-  cluster.sync();
-  uint32_t ties_before = 0, out_before = 0;
-  for (int r = 0; r < rank; ++r) {
-    const uint32_t* rc = cluster.map_shared_rank(sm.cnt, r);
-    const uint32_t c0 = rc[0], c1 = rc[1];
-    out_before += c0 + min(c1, tie_take > ties_before ? tie_take - ties_before : 0u);
-    ties_before += c1;
-  }
-  const uint32_t ntie = sm.cnt[1];
-  const uint32_t take = min(ntie, tie_take > ties_before ? tie_take - ties_before : 0u);
-
-  // Mark the `take` lowest positions among this CTA's keys equal to K.
-  if (take > 0) {
-    if (ntie <= (uint32_t)kTieCap) {
-      for (uint32_t i = tid; i < ntie; i += blockDim.x) {
-        const uint32_t pos = sm.tie_pos[i];
-        uint32_t below = 0;
-        for (uint32_t j = 0; j < ntie; ++j) below += sm.tie_pos[j] < pos;
-        if (below < take) atomicOr(&bitmap[pos >> 5], 1u << (pos & 31));
-      }
-    } else {
-      // Many ties: rank them in position order (per-warp contiguous word ranges).
-      const int wb = warp * wpw, we = min(nwords, wb + wpw);
-      uint32_t mine = 0;
-      for (int word = wb; word < we; ++word) {
-        const int lr = word * 32 + lane;
-        mine += __popc(__ballot_sync(0xffffffffu, lr < nrows && keys[lr] == K));
-      }
-      uint32_t* wt = sm.scan;
-      __syncthreads();
-      if (lane == 0) wt[warp] = mine;
-      __syncthreads();
-      uint32_t rank_before = 0;
-      for (int w = 0; w < warp; ++w) rank_before += wt[w];
-      for (int word = wb; word < we; ++word) {
-        const int lr = word * 32 + lane;
-        const bool eq = lr < nrows && keys[lr] == K;
-        const uint32_t be = __ballot_sync(0xffffffffu, eq);
-        if (eq && rank_before + __popc(be & lt_mask) < take) atomicOr(&bitmap[word], 1u << lane);
-        rank_before += __popc(be);
-      }
+#pragma unroll
+  for (int k = 0; k < SPT; ++k) {
+    const int j = tid + k * kSampleThreads;
+    if (j < S) {
+      const uint32_t key = score_key(v[k]);
+      skey[j] = key;
+      atomicAdd(&hist[key >> 21], 1u);
     }
   }
   __syncthreads();
-
-  // Emit this CTA's selected positions in ascending order from the bitmap.
-  {
-    const int wpt = (nwords + blockDim.x - 1) / blockDim.x;
-    const int wb = tid * wpt, we = min(nwords, wb + wpt);
-    uint32_t mine = 0;
-    for (int word = wb; word < we; ++word) mine += __popc(bitmap[word]);
-    uint32_t slot = out_before + block_exclusive_scan(mine, sm.scan, nullptr);
-    for (int word = wb; word < we; ++word) {
-      uint32_t bits = bitmap[word];
-      while (bits) {
-        const int bit = __ffs(bits) - 1;
-        bits &= bits - 1;
-        if (slot < (uint32_t)p.M) idx_out[slot] = t_begin + word * 32 + bit;
-        ++slot;
-      }
-    }
-  }
-  if (rank == 0 && tid == 0) p.count[(size_t)b * p.Hkv + h] = p.M;
-  cluster.sync();  // no CTA leaves while another may still read its counters
+  const uint32_t tau = sample_threshold<kSampleThreads>(hist, skey, S, n, p.M, scan, digit);
+  if (tid == 0) p.tau[bh] = tau;
 }
+
+constexpr int kFilterChunk = 4096;   // positions per filter CTA
+constexpr int kFilterThreads = 128;  // 4 warps, 1024 positions each
+
+// Per 4096-position chunk of (b, KV head): every position whose key reaches the threshold is
+// appended to the pair's candidate buffer.  Each warp reads its 1024 scores (coalesced, all in
+// flight before the threshold is awaited: the scores are inputs of the call), compacts the keys
+// above the threshold with warp ballots into a shared-memory stage, and flushes the stage with one
+// global atomic when it would overflow and at the end.
+__global__ void __launch_bounds__(kFilterThreads) lisa_select_filter_kernel(IndexParams p) {
+  constexpr int WARPS = kFilterThreads / 32;
+  constexpr int WROWS = kFilterChunk / WARPS;
+  constexpr int PL = WROWS / 32;  // scores per lane
+  __shared__ uint2 cstage[WARPS][kWarpStage];
+  const int h = blockIdx.y, b = blockIdx.z, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const size_t bh = (size_t)b * p.Hkv + h;
+  const int t_begin = blockIdx.x * kFilterChunk;
+  const int n = load_seq_len(p, b);
+  if (n <= p.M || t_begin >= n) {
+    pdl_wait();  // no CTA ends before the earlier kernels of the stream have completed
+    return;
+  }
+  const int w0 = t_begin + warp * WROWS;    // first position of this warp
+  const int wend = min(n, w0 + WROWS);      // one past its last
+  const float* sc = p.scores + bh * (size_t)p.max_seq_len;
+  float v[PL];
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const int t = w0 + 32 * k + lane;
+    v[k] = t < wend ? __ldg(sc + t) : 0.f;
+  }
+  pdl_wait();  // the threshold comes from the sample kernel
+  pdl_trigger();
+  const uint32_t tau = p.tau[bh];
+  uint32_t wn = 0u;  // candidates staged by this warp (the same in every lane)
+  uint2* cdst = reinterpret_cast<uint2*>(p.cand) + bh * (size_t)p.cap;
+  auto flush = [&]() {
+    __syncwarp();
+    if (wn == 0u) return;
+    uint32_t base = 0u;
+    if (lane == 0) base = atomicAdd(&p.ccount[bh], wn);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    for (uint32_t i = lane; i < wn; i += 32u) {
+      const uint32_t slot = base + i;
+      if (slot < (uint32_t)p.cap) cdst[slot] = cstage[warp][i];
+    }
+    __syncwarp();
+  };
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < PL; ++k) {
+    const int t = w0 + 32 * k + lane;
+    const uint32_t key = score_key(v[k]);
+    const bool keep = t < wend && key >= tau;
+    const uint32_t ballot = __ballot_sync(0xffffffffu, keep);
+    if (ballot != 0u) {
+      const uint32_t tot = (uint32_t)__popc(ballot);
+      if (wn + tot > (uint32_t)kWarpStage) {
+        flush();
+        wn = 0u;
+      }
+      if (keep) cstage[warp][wn + __popc(ballot & below)] = make_uint2(key, (uint32_t)t);
+      wn += tot;
+    }
+  }
+  flush();
+}
+
+}  // namespace
+
 
 
 constexpr int kFinishThreads = 512;
-constexpr uint32_t kFinishStageCap = 16384;  // candidates the finish kernel stages in shared memory
-
-__host__ __device__ static uint32_t finish_stage_cap(int cap) { return (uint32_t)cap < kFinishStageCap ? (uint32_t)cap : kFinishStageCap; }
+// Candidates the finish kernel stages in shared memory: about twice the expected count (4M, the
+// threshold aims at 2M), between 8192 (two CTAs per SM still fit at 128K context) and 16384; a pair
+// with more candidates reads them from global memory in each pass.
+__host__ __device__ static uint32_t finish_stage_cap(int cap, int M) {
+  const uint32_t want = (uint32_t)min(max(4 * M, 8192), 16384);
+  return (uint32_t)cap < want ? (uint32_t)cap : want;
+}
 // Words of one position bitmap, rounded up to even so that the candidate stage is 16-byte aligned.
 __host__ __device__ static int finish_bitmap_words(int max_seq_len) { return ((max_seq_len + 63) / 64) * 2; }
 
-size_t finish_smem_bytes(int max_seq_len, int cap) {
-  return (size_t)2 * finish_bitmap_words(max_seq_len) * 4 + (size_t)finish_stage_cap(cap) * 8;
+size_t finish_smem_bytes(int max_seq_len, int cap, int M) {
+  return (size_t)2 * finish_bitmap_words(max_seq_len) * 4 + (size_t)finish_stage_cap(cap, M) * 8;
 }
 
-// One CTA per (KV head, sequence) with n > M: exact top-M from the streamed candidates.
-template <int R, bool FP8>
+// One CTA per (KV head, sequence) with n > M: exact top-M from the streamed candidates (the exact
+// fallback re-scores the projected keys, or reads the caller's scores when FROM_SCORES).
+template <int R, bool FP8, bool FROM_SCORES>
 __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(IndexParams p) {
   extern __shared__ __align__(16) uint32_t fsm[];
   const int h = blockIdx.x, b = blockIdx.y;
@@ -1197,7 +1074,7 @@ __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(Index
   pdl_trigger();
   if (n <= p.M) return;  // the sample kernel wrote the full set
   uint32_t* cstage = fsm + 2 * finish_bitmap_words(p.max_seq_len);
-  finish_pair<R, FP8, kFinishThreads>(p, b, h, n, fsm, cstage, finish_stage_cap(p.cap));
+  finish_pair<R, FP8, kFinishThreads, FROM_SCORES>(p, b, h, n, fsm, cstage, finish_stage_cap(p.cap, p.M));
 }
 
 
@@ -1211,13 +1088,17 @@ static cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream) {
-  (void)from_scores;
-  const size_t smem = select_smem_bytes(p.chunk_max, p.ps);
-  cudaError_t e = set_smem(lisa_select_from_scores_kernel, smem);
+cudaError_t launch_index_select(const IndexParams& p, cudaStream_t stream) {
+  cudaError_t e = launch_pdl(lisa_select_sample_kernel, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
-  lisa_select_from_scores_kernel<<<dim3(kClusterSize, p.Hkv, p.B), kIndexThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  const dim3 grid((p.max_seq_len + kFilterChunk - 1) / kFilterChunk, p.Hkv, p.B);
+  e = launch_pdl(lisa_select_filter_kernel, grid, dim3(kFilterThreads), 0, stream, p);
+  if (e != cudaSuccess) return e;
+  const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap, p.M);
+  auto f = lisa_index_finish_kernel<32, true, true>;
+  e = set_smem(f, fs);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);
 }
 
 template <int R, bool FP8>
@@ -1235,8 +1116,8 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
   e = launch_pdl(k, grid, dim3(kStreamThreads), ring, stream, p);
   if (e != cudaSuccess) return e;
   if (after_stream != nullptr && (e = cudaEventRecord(after_stream, stream)) != cudaSuccess) return e;
-  const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap);
-  auto f = lisa_index_finish_kernel<R, FP8>;
+  const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap, p.M);
+  auto f = lisa_index_finish_kernel<R, FP8, false>;
   e = set_smem(f, fs);
   if (e != cudaSuccess) return e;
   return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);

@@ -13,7 +13,6 @@ constexpr int kSampleMax = 4096;    // positions the threshold sample scores per
 
 struct IndexParams {
   int B, Hq, Hkv, d, r, M, ps, log2ps, max_pages, max_seq_len, num_pages;
-  int chunk_max;  // positions per CTA of a select cluster, at most (multiple of ps)
   int cap;        // candidate-buffer entries per (b, KV head)
   bool kproj_fp8;
   float* uq;           // [B][Hkv][32]: projected averaged query (written by the sample kernel)
@@ -27,7 +26,7 @@ struct IndexParams {
   const float* P;
   const void* kproj;
   const float* kproj_scale;
-  float* scores;  // written by the score kernel, read by the select-from-scores kernel
+  float* scores;  // written by the score kernel, read by the select-from-scores kernels
   int32_t* idx;
   int32_t* count;
   uint32_t* err;
@@ -117,11 +116,10 @@ struct AttnParams {
 };
 
 
-size_t select_smem_bytes(int chunk_max, int ps);
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
-cudaError_t launch_index_select(const IndexParams& p, bool from_scores, cudaStream_t stream);
+cudaError_t launch_index_select(const IndexParams& p, cudaStream_t stream);
 // Launch with programmatic stream serialization (the kernel must call pdl_wait before it touches
 // memory an earlier kernel of the stream may write).
 template <typename... KArgs, typename... Args>
@@ -150,7 +148,7 @@ inline cudaError_t prefer_max_smem(void (*kernel)(KArgs...)) {
 // after_sample / after_stream: optional events recorded between the three kernels (nullptr: none).
 cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample = nullptr,
                               cudaEvent_t after_stream = nullptr);
-size_t finish_smem_bytes(int max_seq_len, int cap);
+size_t finish_smem_bytes(int max_seq_len, int cap, int M);
 cudaError_t launch_sparse_attn(const AttnParams& p, cudaStream_t stream);
 cudaError_t launch_gather(const GatherParams& p, cudaStream_t stream);
 cudaError_t launch_calibrate(const CalibParams& p, cudaStream_t stream);

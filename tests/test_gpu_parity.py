@@ -92,6 +92,8 @@ SELECT_CASES = [
     ([9000, 4100], 2, 300, "ties"),
     ([6000], 2, 1000, "all_equal"),
     ([30000, 12345], 2, 2048, "coarse"),
+    ([20000], 2, 1000, "all_equal"),      # more equal keys than the candidate buffer holds
+    ([100000, 3000], 1, 2048, "hot_sampled"),  # high scores only where the threshold sample looks
 ]
 
 
@@ -112,6 +114,12 @@ def test_topm_select_bit_exact(cuda_device, lens, Hkv, M, mode):
             elif mode == "coarse":
                 v = np.round(v, 1).astype(np.float32)
                 v[rng.choice(n, 5, replace=False)] = -0.0
+            elif mode == "hot_sampled" and n > 4096:
+                # 300 of the sampled positions (runs of 8, one run every n / 512 positions) score far
+                # above the rest: the sampled threshold sits above the M-th score, fewer than M
+                # candidates pass, and the exact path over all scores runs.
+                hot = np.array([(j // 8) * n // 512 + j % 8 for j in range(300)])
+                v[hot] = 100.0 + rng.random(300).astype(np.float32)
             s[b, h, :n] = v
     table, kw = _select_desc(B, Hkv, M, max_len, cuda_device)
     seq = torch.tensor(lens, dtype=torch.int32, device=cuda_device)
