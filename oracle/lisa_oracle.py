@@ -386,5 +386,6 @@ def multi_query_scores(inp: dict, q_tokens, T: int, b: int, h: int) -> np.ndarra
         one["q"] = np.asarray(q_tokens)[:, j]  # [B][Hq][d]: token j of every sequence
         s = head_scores(one, b, h)
         lim = n - T + j
-        out[j, : lim + 1] = s[: lim + 1]
+        if lim >= 0:  # a token of a sequence shorter than T may see no position at all
+            out[j, : lim + 1] = s[: lim + 1]
     return out

@@ -540,6 +540,20 @@ def test_multi_query_scores_are_single_queries_over_causal_prefixes():
                 assert np.all(np.isneginf(s[j, n - T + j + 1 :]))
 
 
+def test_multi_query_tokens_of_a_short_sequence_see_only_their_prefix():
+    # n = 2 positions, T = 4 tokens: tokens 0 and 1 see nothing, token 2 sees position 0, token 3 both
+    prob = make_problem(name="mq", B=1, Hq=4, Hkv=1, d=64, r=16, M=4, seq_lens=[2], page_size=16, paged=False,
+                        kproj_fp8=True, plant=("none",), seed=32, device=torch.device("cpu"))
+    inp = host_inputs(prob)
+    rng = np.random.default_rng(33)
+    qt = _bf16_bits(rng.normal(size=(1, 4, prob.Hq, prob.d)))
+    s = O.multi_query_scores(inp, qt, 4, 0, 0)
+    assert s.shape == (4, 2)
+    assert np.all(np.isneginf(s[0])) and np.all(np.isneginf(s[1]))
+    assert np.isfinite(s[2, 0]) and np.isneginf(s[2, 1])
+    assert np.all(np.isfinite(s[3]))
+
+
 def test_mutations_are_caught(monkeypatch):
     good_project, good_select, good_attn = O.project_query, O.select_top_m, O.sparse_attention
     good_gate, good_upd = O.gate_combine, O.linear_state_update
