@@ -167,6 +167,23 @@ lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens,
                                    const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
                                    float* scores, void* ws, size_t ws_bytes, lisa_stream_t stream);
 
+/* Workspace bytes lisa_index_topm_multi needs for `desc` and T = num_tokens (those of a desc with
+ * B * T sequences; 0 if desc or num_tokens is invalid). Host only. */
+size_t lisa_workspace_size_multi(const lisa_decode_desc* desc, int num_tokens);
+
+/* Steps 1-4 fused for T query tokens per sequence (1 <= T <= 8, B * T <= 65535), FP8 projected keys
+ * only: token j of sequence b (q bf16 [B][T][Hq][d]) averages its G queries per KV head, projects
+ * them with P_h and keeps the min(M, n_b - T + j + 1) best of the positions t <= n_b - T + j (ties to
+ * the lower position), ascending, in idx int32 [B][T][Hkv][M] (the rest -1) with count int32
+ * [B][T][Hkv].  The same sets as lisa_index_score_multi followed by lisa_topm_select on a desc of
+ * B * T sequences, without writing the scores: a sampled threshold per token, one stream of the
+ * projected keys for all T tokens (the per-tile tensor-core contraction of lisa_index_score_multi)
+ * that keeps each token's positions above its threshold, and the exact finish per token (with the
+ * same exact re-scoring fallback as lisa_index_topm).  ws: lisa_workspace_size_multi bytes. */
+lisa_status lisa_index_topm_multi(const lisa_decode_desc* desc, int num_tokens, const void* q, const float* P,
+                                  const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
+                                  int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, lisa_stream_t stream);
+
 /* Step 4 from caller-given fp32 scores: idx[b][h][0..count) ascending, count = min(M, n_b),
  * idx[b][h][count..M) = -1. */
 lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx,

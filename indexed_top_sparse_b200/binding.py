@@ -106,6 +106,8 @@ _sig = {
     "lisa_dense_workspace_size": (ctypes.c_size_t, [ctypes.POINTER(DecodeDesc)]),
     "lisa_calibrate_workspace_size": (ctypes.c_size_t, [_I, _I]),
     "lisa_index_score_multi": (_I, [ctypes.POINTER(DecodeDesc), _I, _P, _P, _P, _I, _P, _P, _P, _S, _P]),
+    "lisa_workspace_size_multi": (ctypes.c_size_t, [ctypes.POINTER(DecodeDesc), _I]),
+    "lisa_index_topm_multi": (_I, [ctypes.POINTER(DecodeDesc), _I, _P, _P, _P, _I, _P, _P, _P, _P, _S, _P]),
     "lisa_calibrate_basis": (_I, [_I, _I, _I, _P, _I, _P, _I, _P, _P, _P, _S, _P]),
     "lisa_dense_decode_attn": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
     "lisa_gather_kv": (_I, [ctypes.POINTER(DecodeDesc), _P, _P, _P, _P, _P, _P, _S, _P]),
@@ -294,6 +296,29 @@ def lisa_index_score_multi(desc, num_tokens, q, P, kproj_pool, kproj_dtype, kpro
         _lib.lisa_index_score_multi(ctypes.byref(desc), num_tokens, _ptr(q), _ptr(P), _ptr(kproj_pool), kproj_dtype,
                                     _ptr(kproj_scale), _ptr(scores), _ptr(ws), ws.numel(), _stream(stream)),
         "lisa_index_score_multi",
+    )
+
+
+def lisa_workspace_size_multi(desc, num_tokens: int) -> int:
+    return int(_lib.lisa_workspace_size_multi(ctypes.byref(desc), num_tokens))
+
+
+def alloc_workspace_multi(desc: DecodeDesc, num_tokens: int, device, stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for lisa_index_topm_multi."""
+    n = lisa_workspace_size_multi(desc, num_tokens)
+    if n == 0:
+        raise LisaError(1, "lisa_workspace_size_multi")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    lisa_workspace_init(ws, stream)
+    return ws
+
+
+def lisa_index_topm_multi(desc, num_tokens, q, P, kproj_pool, kproj_dtype, kproj_scale, idx, count, ws,
+                          stream=None) -> None:
+    _check(
+        _lib.lisa_index_topm_multi(ctypes.byref(desc), num_tokens, _ptr(q), _ptr(P), _ptr(kproj_pool), kproj_dtype,
+                                   _ptr(kproj_scale), _ptr(idx), _ptr(count), _ptr(ws), ws.numel(), _stream(stream)),
+        "lisa_index_topm_multi",
     )
 
 

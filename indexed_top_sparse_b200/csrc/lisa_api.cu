@@ -170,6 +170,7 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   p.max_seq_len = d.max_seq_len;
   p.num_pages = d.num_pages;
   p.cap = L.cap;
+  p.T = 1;
   p.seq_lens = d.seq_lens;
   p.page_table = d.page_table;
   p.err = static_cast<uint32_t*>(ws);
@@ -305,6 +306,13 @@ size_t lisa_workspace_size(const lisa_decode_desc* desc) {
   return layout_of(*desc).total;
 }
 
+size_t lisa_workspace_size_multi(const lisa_decode_desc* desc, int num_tokens) {
+  if (check_desc(desc) != LISA_OK || num_tokens < 1 || num_tokens > kMultiMaxT) return 0;
+  lisa_decode_desc d = *desc;
+  d.batch = desc->batch * num_tokens;
+  return layout_of(d).total;
+}
+
 int32_t lisa_num_splits(const lisa_decode_desc* desc) {
   if (check_desc(desc) != LISA_OK) return 0;
   return layout_of(*desc).splits;
@@ -376,6 +384,62 @@ lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens,
   p.uq = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.off_cand);
   p.err = static_cast<uint32_t*>(ws);
   return cuda_status(launch_index_score_multi(p, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+lisa_status lisa_index_topm_multi(const lisa_decode_desc* desc, int num_tokens, const void* q, const float* P,
+                                  const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
+                                  int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, lisa_stream_t stream) {
+  LISA_TRY(check_desc(desc));
+  if (desc->batch == 0) return LISA_OK;
+  LISA_TRY(check_idx_dim(desc));
+  if (num_tokens < 1 || num_tokens > kMultiMaxT) return LISA_ERR_UNSUPPORTED;
+  if (kproj_dtype != LISA_KPROJ_FP8_E4M3) return LISA_ERR_UNSUPPORTED;
+  if ((long long)desc->batch * num_tokens > 65535) return LISA_ERR_UNSUPPORTED;
+  if (q == nullptr || P == nullptr || kproj_pool == nullptr || kproj_scale == nullptr || idx == nullptr ||
+      count == nullptr)
+    return LISA_ERR_INVALID_ARG;
+  if (!aligned32(kproj_pool) || !aligned4(q) || !aligned4(P)) return LISA_ERR_INVALID_ARG;
+  // Index rows (b * T + j, h): the workspace of a desc with B * T sequences.
+  lisa_decode_desc dbt = *desc;
+  dbt.batch = desc->batch * num_tokens;
+  const Layout L = layout_of(dbt);
+  LISA_TRY(check_ws(ws, ws_bytes, L));
+  LISA_TRY(bind_device(ws));
+  IndexParams p = index_params(dbt, L, ws);
+  p.T = num_tokens;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.P = P;
+  p.kproj = kproj_pool;
+  p.kproj_fp8 = true;
+  p.kproj_scale = kproj_scale;
+  p.idx = idx;
+  p.count = count;
+  MultiParams m{};
+  m.B = desc->batch;
+  m.T = num_tokens;
+  m.Hq = desc->num_q_heads;
+  m.Hkv = desc->num_kv_heads;
+  m.d = desc->head_dim;
+  m.r = desc->idx_dim;
+  m.ps = desc->page_size;
+  m.log2ps = ilog2(desc->page_size);
+  m.max_pages = desc->max_pages_per_seq;
+  m.max_seq_len = desc->max_seq_len;
+  m.num_pages = desc->num_pages;
+  m.seq_lens = desc->seq_lens;
+  m.page_table = desc->page_table;
+  m.q = p.q;
+  m.P = P;
+  m.kproj = kproj_pool;
+  m.kproj_scale = kproj_scale;
+  m.uq = p.uq;
+  m.err = p.err;
+  m.M = p.M;
+  m.cap = p.cap;
+  m.tau = p.tau;
+  m.ccount = p.ccount;
+  m.cand = p.cand;
+  return cuda_status(launch_index_topm_multi(p, m, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx, int32_t* count,

@@ -168,6 +168,13 @@ __device__ __forceinline__ int load_seq_len(const IndexParams& p, int b) {
   return n;
 }
 
+// Context seen by index row bj.  With T query tokens per sequence, row bj is token j = bj % T of
+// sequence bj / T, which sees the positions t <= n - T + j.
+__device__ __forceinline__ int load_pair_len(const IndexParams& p, int bj) {
+  if (p.T == 1) return load_seq_len(p, bj);
+  return max(0, load_seq_len(p, bj / p.T) - (p.T - 1 - bj % p.T));
+}
+
 // qbar = mean of the G query rows of KV head h; u = P_h qbar.  Ends with a barrier.
 __device__ void compute_projected_query(const IndexParams& p, int b, int h, float* qbar, float* u) {
   const int G = p.Hq / p.Hkv;
@@ -405,7 +412,8 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
   const size_t bh = (size_t)b * p.Hkv + h;
   pdl_wait();  // first kernel of the step: everything it reads may come from earlier stream work
   pdl_trigger();
-  const int n = load_seq_len(p, b);
+  const int n = load_pair_len(p, b);
+  const int bs = p.T == 1 ? b : b / p.T;  // the sequence whose cache row b reads
   const int G = p.Hq / p.Hkv;
   const int S = min(n, kSampleMax);
   const bool sampling = n > p.M;
@@ -435,7 +443,7 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
     const int j = tid + k * kSampleThreads;
     pg[k] = 0;
     tpos[k] = sample_pos(j, n);
-    if (sampling && j < S) pg[k] = p.page_table[(size_t)b * p.max_pages + (tpos[k] >> p.log2ps)];
+    if (sampling && j < S) pg[k] = p.page_table[(size_t)bs * p.max_pages + (tpos[k] >> p.log2ps)];
   }
   for (int i = tid; i < kBins; i += blockDim.x) hist[i] = 0u;
   if (tid < p.d) qbar[tid] = qsum / (float)G;
@@ -591,7 +599,7 @@ __device__ void finish_pair(const IndexParams& p, int b, int h, int n, uint32_t*
     } else {
       for (int t = tid; t < n; t += blockDim.x) {
         uint32_t w[RowGeom<R, FP8>::kWords];
-        load_row<R, FP8>(p, b, h, t, w);
+        load_row<R, FP8>(p, p.T == 1 ? b : b / p.T, h, t, w);
         fn(score_key(scale * row_dot<R, FP8>(w, u2)), (uint32_t)t);
       }
     }
@@ -1069,7 +1077,7 @@ template <int R, bool FP8, bool FROM_SCORES>
 __global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(IndexParams p) {
   extern __shared__ __align__(16) uint32_t fsm[];
   const int h = blockIdx.x, b = blockIdx.y;
-  const int n = load_seq_len(p, b);
+  const int n = load_pair_len(p, b);
   pdl_wait();  // candidates and counts come from the streaming kernel
   pdl_trigger();
   if (n <= p.M) return;  // the sample kernel wrote the full set
@@ -1121,6 +1129,25 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
   e = set_smem(f, fs);
   if (e != cudaSuccess) return e;
   return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);
+}
+
+// Fused multi-query top-M: sample and finish over the B*T index rows, and between them one stream
+// of the projected keys for all T tokens of each sequence.
+template <int R>
+static cudaError_t launch_topm_multi_t(const IndexParams& p, const MultiParams& m, cudaStream_t stream) {
+  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
+  if (e != cudaSuccess) return e;
+  e = launch_index_topm_multi_stream(m, stream);
+  if (e != cudaSuccess) return e;
+  const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap, p.M);
+  auto f = lisa_index_finish_kernel<R, true, false>;
+  e = set_smem(f, fs);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);
+}
+
+cudaError_t launch_index_topm_multi(const IndexParams& p, const MultiParams& m, cudaStream_t stream) {
+  return p.r == 16 ? launch_topm_multi_t<16>(p, m, stream) : launch_topm_multi_t<32>(p, m, stream);
 }
 
 cudaError_t launch_index_topm(const IndexParams& p, cudaStream_t stream, cudaEvent_t after_sample,

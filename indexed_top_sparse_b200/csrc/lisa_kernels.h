@@ -14,6 +14,7 @@ constexpr int kSampleMax = 4096;    // positions the threshold sample scores per
 struct IndexParams {
   int B, Hq, Hkv, d, r, M, ps, log2ps, max_pages, max_seq_len, num_pages;
   int cap;        // candidate-buffer entries per (b, KV head)
+  int T;          // query tokens per sequence: index row b is token b % T of sequence b / T (1: decode)
   bool kproj_fp8;
   float* uq;           // [B][Hkv][32]: projected averaged query (written by the sample kernel)
   uint32_t* tau;       // [B][Hkv]: candidate threshold key
@@ -82,6 +83,11 @@ struct MultiParams {
   float* scores;           // [B][T][Hkv][max_seq_len]
   float* uq;               // workspace: projected queries [B][T][Hkv][32]
   uint32_t* err;
+  // Fused per-token top-M only: rows (b * T + j, h) of the index workspace.
+  int M, cap;
+  const uint32_t* tau;     // [B*T][Hkv] candidate threshold keys
+  uint32_t* ccount;        // [B*T][Hkv]
+  uint32_t* cand;          // [B*T][Hkv][cap][2]
 };
 
 struct AttnParams {
@@ -118,6 +124,10 @@ struct AttnParams {
 
 size_t attn_smem_bytes(int d);
 cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream);
+// Candidate stream of the fused multi-query top-M (between the sample and finish kernels).
+cudaError_t launch_index_topm_multi_stream(const MultiParams& p, cudaStream_t stream);
+// The fused multi-query top-M: p indexes the B*T rows (p.T = T), m streams the B sequences.
+cudaError_t launch_index_topm_multi(const IndexParams& p, const MultiParams& m, cudaStream_t stream);
 cudaError_t launch_index_score(const IndexParams& p, cudaStream_t stream);
 cudaError_t launch_index_select(const IndexParams& p, cudaStream_t stream);
 // Launch with programmatic stream serialization (the kernel must call pdl_wait before it touches

@@ -30,6 +30,7 @@ constexpr int kMultiThreads = 128;      // 4 warps, 1024 positions each
 constexpr int kMultiStageBytes = 2048;  // projected-key bytes per warp pipeline stage
 constexpr int kMultiStages = 4;         // stages in each warp's shared-memory ring
 constexpr int kMultiCtasPerSm = 6;
+constexpr int kMultiTopmStage = 64;    // candidates a warp stages per query between flushes
 
 // uq[b][j][h][0..r): the projected mean query of token j (fp32, 32 slots per row).
 __global__ void __launch_bounds__(kMultiThreads) lisa_multi_project_kernel(MultiParams p) {
@@ -77,9 +78,12 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_multi_project_kernel(Multi
   }
 }
 
-template <int R, int NT>
+// TOPM = false: the scores of every visible (token, position) are written.  TOPM = true: nothing is
+// written but the positions whose key reaches their token's sampled threshold, appended to that
+// token's candidate buffer (staged per warp and token in shared memory, behind the ring).
+template <int R, int NT, bool TOPM>
 __global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_multi_kernel(MultiParams p) {
-  extern __shared__ __align__(128) uint8_t ring[];   // [warp][kMultiStages][kMultiStageBytes]
+  extern __shared__ __align__(128) uint8_t ring[];   // [warp][kMultiStages][kMultiStageBytes], then the stage
   __shared__ const uint8_t* pbase[kMultiChunk / 16];  // global address of each page block of the chunk
   __shared__ float ush[kMultiMaxT][32];
   constexpr int RB = R;                        // FP8: one byte per dimension
@@ -196,15 +200,50 @@ __global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_mul
       for (int i = 0; i < R; ++i) mo = fmaxf(mo, fabsf(ush[jo][i]));
     const int Eo = mo > 0.f ? ilogbf(mo) - 13 : 0;
     fac[nt] = p.kproj_scale[h] * ldexpf(1.f, Eo);
-    srow[nt] = p.scores + (((size_t)b * T + min(jo, T - 1)) * p.Hkv + h) * p.max_seq_len + t_begin + w0;
+    if constexpr (!TOPM)
+      srow[nt] = p.scores + (((size_t)b * T + min(jo, T - 1)) * p.Hkv + h) * p.max_seq_len + t_begin + w0;
   }
-  // lim[nt]: the last warp-relative row query 4 nt + t sees (negative: none).
+  // lim[nt]: the last warp-relative row query 4 nt + t sees (negative: none).  A token whose context
+  // is at most M positions long has its full set from the sample kernel and takes no candidates.
   int lim[NT];
+  uint32_t tau[NT];         // candidate threshold key of query 4 nt + t
+  uint2* cdst[NT];          // its candidate buffer
+  uint32_t* ccnt[NT];       // and count
+  uint32_t wn[NT];          // candidates of that query staged by this warp (same in its 8 lanes)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int jo = 4 * nt + t4;
-    lim[nt] = jo < T ? min(n - T + jo - t_begin - w0, wrows - 1) : -1;
+    bool live = jo < T;
+    if constexpr (TOPM) live = live && n - T + jo + 1 > p.M;
+    lim[nt] = live ? min(n - T + jo - t_begin - w0, wrows - 1) : -1;
+    if constexpr (TOPM) {
+      const size_t pair = ((size_t)b * T + min(jo, T - 1)) * p.Hkv + h;
+      tau[nt] = live ? p.tau[pair] : 0xffffffffu;
+      cdst[nt] = reinterpret_cast<uint2*>(p.cand) + pair * (size_t)p.cap;
+      ccnt[nt] = p.ccount + pair;
+      wn[nt] = 0u;
+    }
   }
+  // Per-(warp, query) stages of kMultiTopmStage (key, position) entries, behind the ring.
+  uint2* wstage = reinterpret_cast<uint2*>(ring + (kMultiThreads / 32) * kMultiStages * kMultiStageBytes) +
+                  (size_t)warp * (4 * NT) * kMultiTopmStage;
+  // Appends the staged candidates of the four queries of n-tile nt (lane group t of the warp owns
+  // query 4 nt + t) to their buffers, one global atomic per query; entries past the capacity are
+  // dropped and the count then sends that query to the exact path.
+  auto flush = [&](int nt) {
+    __syncwarp();
+    const uint32_t cnt = wn[nt];
+    uint32_t base = 0u;
+    if (g == 0 && cnt > 0u) base = atomicAdd(ccnt[nt], cnt);
+    base = __shfl_sync(0xffffffffu, base, t4);
+    const uint2* st_q = wstage + (size_t)(4 * nt + t4) * kMultiTopmStage;
+    for (uint32_t i = g; i < cnt; i += 8u) {
+      const uint32_t slot = base + i;
+      if (slot < (uint32_t)p.cap) cdst[nt][slot] = st_q[i];
+    }
+    wn[nt] = 0u;
+    __syncwarp();
+  };
 
   for (int st = 0; st < nstages; ++st) {
     issue(st + kMultiStages - 1);
@@ -212,8 +251,15 @@ __global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_mul
     cp_async_wait<kMultiStages - 1>();
     __syncwarp();
     const uint8_t* src = wring + (st % kMultiStages) * kMultiStageBytes;
+    // Tiles in groups of four (64 rows); with TOPM the group's candidates are staged after it.
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+    for (int mg = 0; mg < MT; mg += 4) {
+    uint32_t keys[NT][8];
+    uint32_t mask[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) mask[nt] = 0u;
+#pragma unroll
+    for (int mt = mg; mt < mg + 4; ++mt) {
       const uint8_t* r0 = src + (mt * 16 + g) * RB + (R / 4) * t4;
       const uint8_t* r1 = r0 + 8 * RB;
       uint32_t x0[KS], x1[KS];
@@ -243,22 +289,64 @@ __global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_mul
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int rr = st * RPS + mt * 16 + g;
-        if (rr <= lim[nt]) srow[nt][rr] = fac[nt] * (dacc[nt][0] + dacc[nt][1]);
-        if (rr + 8 <= lim[nt]) srow[nt][rr + 8] = fac[nt] * (dacc[nt][2] + dacc[nt][3]);
+        const float s0 = fac[nt] * (dacc[nt][0] + dacc[nt][1]), s1 = fac[nt] * (dacc[nt][2] + dacc[nt][3]);
+        if constexpr (TOPM) {
+          const int k = 2 * (mt - mg);
+          keys[nt][k] = score_key(s0);
+          keys[nt][k + 1] = score_key(s1);
+          if (rr <= lim[nt] && keys[nt][k] >= tau[nt]) mask[nt] |= 1u << k;
+          if (rr + 8 <= lim[nt] && keys[nt][k + 1] >= tau[nt]) mask[nt] |= 2u << k;
+        } else {
+          if (rr <= lim[nt]) srow[nt][rr] = s0;
+          if (rr + 8 <= lim[nt]) srow[nt][rr + 8] = s1;
+        }
       }
+    }
+    if constexpr (TOPM) {
+      // Slots from a prefix sum over the 8 lanes that hold the same query (lanes t, t + 4, ...).
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint32_t c = (uint32_t)__popc(mask[nt]);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, incl, 28 + t4);
+        if (__any_sync(0xffffffffu, wn[nt] + tot > (uint32_t)kMultiTopmStage)) flush(nt);
+        uint32_t slot = wn[nt] + incl - c;
+        uint2* st_q = wstage + (size_t)(4 * nt + t4) * kMultiTopmStage;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if ((mask[nt] >> k) & 1u) {
+            const int row = st * RPS + (mg + (k >> 1)) * 16 + g + 8 * (k & 1);
+            st_q[slot++] = make_uint2(keys[nt][k], (uint32_t)(t_begin + w0 + row));
+          }
+        }
+        wn[nt] += tot;
+      }
+    }
     }
     __syncwarp();  // the slot is refilled by a later stage
   }
   cp_async_wait<0>();
+  if constexpr (TOPM) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) flush(nt);
+  }
 }
 
-template <int R, int NT>
+template <int R, int NT, bool TOPM>
 cudaError_t launch_score_multi_t(const MultiParams& p, cudaStream_t stream) {
-  const size_t smem = (size_t)(kMultiThreads / 32) * kMultiStages * kMultiStageBytes;
+  size_t smem = (size_t)(kMultiThreads / 32) * kMultiStages * kMultiStageBytes;
+  if (TOPM) smem += (size_t)(kMultiThreads / 32) * (4 * NT) * kMultiTopmStage * sizeof(uint2);
   const dim3 grid((p.max_seq_len + kMultiChunk - 1) / kMultiChunk, p.Hkv, p.B);
-  cudaError_t e = prefer_max_smem(lisa_score_multi_kernel<R, NT>);
+  auto k = lisa_score_multi_kernel<R, NT, TOPM>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess) e = prefer_max_smem(k);
   if (e != cudaSuccess) return e;
-  return launch_pdl(lisa_score_multi_kernel<R, NT>, grid, dim3(kMultiThreads), smem, stream, p);
+  return launch_pdl(k, grid, dim3(kMultiThreads), smem, stream, p);
 }
 
 }  // namespace
@@ -267,8 +355,16 @@ cudaError_t launch_index_score_multi(const MultiParams& p, cudaStream_t stream) 
   cudaError_t e = launch_pdl(lisa_multi_project_kernel, dim3(p.Hkv, p.B), dim3(kMultiThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
   const bool two = 2 * p.T > 8;  // 2T columns: one or two n-tiles of 8
-  if (p.r == 16) return two ? launch_score_multi_t<16, 2>(p, stream) : launch_score_multi_t<16, 1>(p, stream);
-  return two ? launch_score_multi_t<32, 2>(p, stream) : launch_score_multi_t<32, 1>(p, stream);
+  if (p.r == 16)
+    return two ? launch_score_multi_t<16, 2, false>(p, stream) : launch_score_multi_t<16, 1, false>(p, stream);
+  return two ? launch_score_multi_t<32, 2, false>(p, stream) : launch_score_multi_t<32, 1, false>(p, stream);
+}
+
+cudaError_t launch_index_topm_multi_stream(const MultiParams& p, cudaStream_t stream) {
+  const bool two = 2 * p.T > 8;
+  if (p.r == 16)
+    return two ? launch_score_multi_t<16, 2, true>(p, stream) : launch_score_multi_t<16, 1, true>(p, stream);
+  return two ? launch_score_multi_t<32, 2, true>(p, stream) : launch_score_multi_t<32, 1, true>(p, stream);
 }
 
 }  // namespace lisa
