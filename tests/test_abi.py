@@ -103,6 +103,28 @@ def test_null_and_workspace_checks():
     assert lib.lisa_index_score(ctypes.byref(d), A, A, A, 7, A, A, 0x100, need, None) == 1
 
 
+def test_multi_query_host_checks():
+    d = _desc()
+    lib = B._lib
+    A = 0x1000
+    # the workspace of T tokens is that of a desc with B * T sequences
+    one = L.lisa_workspace_size(d)
+    for T in (1, 2, 4, 8):
+        dt = _desc(batch=d.batch * T)
+        assert L.lisa_workspace_size_multi(d, T) == L.lisa_workspace_size(dt)
+    assert L.lisa_workspace_size_multi(d, 1) == one
+    assert L.lisa_workspace_size_multi(d, 0) == 0 and L.lisa_workspace_size_multi(d, 9) == 0
+    need = L.lisa_workspace_size_multi(d, 4)
+    args = lambda T, kd=1, ws_bytes=need, kproj=A: (ctypes.byref(d), T, A, A, kproj, kd, A, A, A, 0x100, ws_bytes, None)
+    assert lib.lisa_index_topm_multi(*args(9)) == 2       # T > 8
+    assert lib.lisa_index_topm_multi(*args(0)) == 2       # T < 1
+    assert lib.lisa_index_topm_multi(*args(4, kd=0)) == 2  # fp32 projected keys: FP8 only
+    assert lib.lisa_index_topm_multi(*args(4, kproj=A + 16)) == 1  # 32-byte alignment
+    assert lib.lisa_index_topm_multi(*args(4, ws_bytes=need - 1)) == 3
+    assert lib.lisa_index_topm_multi(*args(8, ws_bytes=need)) == 3  # sized for fewer tokens
+    assert lib.lisa_index_score_multi(ctypes.byref(d), 9, A, A, A, 1, A, A, 0x100, one, None) == 2
+
+
 def test_empty_batch_is_a_no_op():
     d = _desc(batch=0)
     d.seq_lens = None
