@@ -397,8 +397,10 @@ __device__ __forceinline__ int sample_pos(int j, int n) {
   return (int)(((uint32_t)(j / kSampleRun) * (uint32_t)n) >> 9) + (j % kSampleRun);
 }
 
-template <int R, bool FP8>
-__global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(IndexParams p) {
+// MINB: CTAs per SM the launch is built for (2 for the B*T index rows of the multi-query top-M,
+// which then loads its sampled rows in two batches).
+template <int R, bool FP8, int MINB = 1>
+__global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel(IndexParams p) {
   __shared__ float qbar[128];
   __shared__ float u[32];
   __shared__ uint32_t hist[kBins];
@@ -450,7 +452,8 @@ __global__ void __launch_bounds__(kSampleThreads) lisa_index_sample_kernel(Index
 
   // Round 2: the sampled rows, KB at a time (all of them for FP8 rows), the first batch in flight
   // while u = P qbar is formed.
-  constexpr int KB = (64 / Geo::kWords) < SPT ? (64 / Geo::kWords) : SPT;
+  constexpr int KB0 = (64 / Geo::kWords) < SPT ? (64 / Geo::kWords) : SPT;
+  constexpr int KB = MINB > 1 && KB0 > 4 ? 4 : KB0;
   uint32_t w[KB][Geo::kWords];
   auto load_batch = [&](int k0) {
 #pragma unroll
@@ -1073,8 +1076,8 @@ size_t finish_smem_bytes(int max_seq_len, int cap, int M) {
 
 // One CTA per (KV head, sequence) with n > M: exact top-M from the streamed candidates (the exact
 // fallback re-scores the projected keys, or reads the caller's scores when FROM_SCORES).
-template <int R, bool FP8, bool FROM_SCORES>
-__global__ void __launch_bounds__(kFinishThreads) lisa_index_finish_kernel(IndexParams p) {
+template <int R, bool FP8, bool FROM_SCORES, int MINB = 1>
+__global__ void __launch_bounds__(kFinishThreads, MINB) lisa_index_finish_kernel(IndexParams p) {
   extern __shared__ __align__(16) uint32_t fsm[];
   const int h = blockIdx.x, b = blockIdx.y;
   const int n = load_pair_len(p, b);
@@ -1135,12 +1138,12 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
 // of the projected keys for all T tokens of each sequence.
 template <int R>
 static cudaError_t launch_topm_multi_t(const IndexParams& p, const MultiParams& m, cudaStream_t stream) {
-  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
+  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true, 2>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
   e = launch_index_topm_multi_stream(m, stream);
   if (e != cudaSuccess) return e;
   const size_t fs = finish_smem_bytes(p.max_seq_len, p.cap, p.M);
-  auto f = lisa_index_finish_kernel<R, true, false>;
+  auto f = lisa_index_finish_kernel<R, true, false, 2>;
   e = set_smem(f, fs);
   if (e != cudaSuccess) return e;
   return launch_pdl(f, dim3(p.Hkv, p.B), dim3(kFinishThreads), fs, stream, p);
