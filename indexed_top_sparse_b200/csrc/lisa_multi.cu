@@ -206,10 +206,10 @@ __global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_mul
   // lim[nt]: the last warp-relative row query 4 nt + t sees (negative: none).  A token whose context
   // is at most M positions long has its full set from the sample kernel and takes no candidates.
   int lim[NT];
-  uint32_t tau[NT];         // candidate threshold key of query 4 nt + t
-  uint2* cdst[NT];          // its candidate buffer
-  uint32_t* ccnt[NT];       // and count
-  uint32_t wn[NT];          // candidates of that query staged by this warp (same in its 8 lanes)
+  uint32_t tau[NT] = {};        // candidate threshold key of query 4 nt + t
+  uint2* cdst[NT] = {};         // its candidate buffer
+  uint32_t* ccnt[NT] = {};      // and count
+  uint32_t wn[NT] = {};         // candidates of that query staged by this warp (same in its 8 lanes)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int jo = 4 * nt + t4;
