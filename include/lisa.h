@@ -184,8 +184,12 @@ lisa_status lisa_index_topm_multi(const lisa_decode_desc* desc, int num_tokens, 
                                   const void* kproj_pool, lisa_kproj_dtype kproj_dtype, const float* kproj_scale,
                                   int32_t* idx, int32_t* count, void* ws, size_t ws_bytes, lisa_stream_t stream);
 
-/* Step 4 from caller-given fp32 scores: idx[b][h][0..count) ascending, count = min(M, n_b),
- * idx[b][h][count..M) = -1. */
+/* Step 4 from caller-given fp32 scores (scores [B][Hkv][max_seq_len], entries t >= n_b never read):
+ * idx[b][h][0..count) ascending, count = min(M, n_b), idx[b][h][count..M) = -1; a tie at the M-th
+ * score goes to the lower position, and -0 equals +0.  Three kernels on `stream`: a threshold
+ * sampled from the scores, a filter that streams the scores and keeps the positions at or above it,
+ * and an exact select over those (over all n_b scores instead when fewer than M pass or the
+ * candidate buffer in ws overflows), so the result is exact whatever the scores. */
 lisa_status lisa_topm_select(const lisa_decode_desc* desc, const float* scores, int32_t* idx,
                              int32_t* count, void* ws, size_t ws_bytes, lisa_stream_t stream);
 
