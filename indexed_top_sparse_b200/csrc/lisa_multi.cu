@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kMultiThreads) lisa_multi_project_kernel(Multi
 // written but the positions whose key reaches their token's sampled threshold, appended to that
 // token's candidate buffer (staged per warp and token in shared memory, behind the ring).
 template <int R, int NT, bool TOPM>
-__global__ void __launch_bounds__(kMultiThreads, kMultiCtasPerSm) lisa_score_multi_kernel(MultiParams p) {
+__global__ void __launch_bounds__(kMultiThreads, TOPM ? kMultiCtasPerSm - 1 : kMultiCtasPerSm) lisa_score_multi_kernel(MultiParams p) {
   extern __shared__ __align__(128) uint8_t ring[];   // [warp][kMultiStages][kMultiStageBytes], then the stage
   __shared__ const uint8_t* pbase[kMultiChunk / 16];  // global address of each page block of the chunk
   __shared__ float ush[kMultiMaxT][32];
