@@ -58,13 +58,24 @@ lisa_status check_idx_dim(const lisa_decode_desc* d) {
 Layout layout_of(const lisa_decode_desc& d) {
   Layout L;
   L.G = d.num_q_heads / d.num_kv_heads;
-  // Stream-K attention: kAttnGrid CTAs (at most one per tile) share the B * Hkv * ceil(M / 64) tiles
-  // evenly; a pair is covered by at most ceil(grid / pairs) + 1 CTAs, each writing one partial.
+  // Stream-K attention: the B * Hkv * ceil(M / 64) tiles are shared evenly by pairs * s CTAs, each
+  // pair cut into s parts.  s is the largest divisor of the tiles per pair that keeps the grid
+  // within kAttnGrid (two CTAs per SM), so that CTA boundaries fall on pair boundaries and no CTA
+  // merges more than one pair; at least ceil(tpp / kAttnMaxTiles) parts, so no CTA takes more than
+  // kAttnMaxTiles tiles (several waves when the pairs alone fill the grid).  A pair is covered by at
+  // most ceil(grid / pairs) + 1 CTAs, each writing one partial.
   L.tpp = (d.budget_m + kAttnTile - 1) / kAttnTile;
   const long long pairs = d.batch > 0 ? (long long)d.batch * d.num_kv_heads : 1;
-  const long long tiles = pairs * L.tpp;
-  long long grid = tiles < kAttnGrid ? tiles : kAttnGrid;
-  if (grid * kAttnMaxTiles < tiles) grid = (tiles + kAttnMaxTiles - 1) / kAttnMaxTiles;
+  const long long s_min = (L.tpp + kAttnMaxTiles - 1) / kAttnMaxTiles;
+  const long long s_cap = pairs < kAttnGrid ? kAttnGrid / pairs : 1;
+  long long s = s_min;
+  for (long long c = s_cap < L.tpp ? s_cap : L.tpp; c > s_min; --c) {
+    if (L.tpp % c == 0) {
+      s = c;
+      break;
+    }
+  }
+  const long long grid = pairs * s;
   L.grid = (int)grid;
   L.splits = (int)((L.grid + pairs - 1) / pairs) + 1;
   const size_t B = (size_t)d.batch, Hkv = (size_t)d.num_kv_heads;
