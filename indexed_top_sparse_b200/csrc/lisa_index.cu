@@ -384,7 +384,7 @@ __device__ uint32_t sample_threshold(uint32_t* hist, const uint32_t* skey, int S
   return (d0 << 21) | (digit[0] << 10);
 }
 
-constexpr int kSampleThreads = 512;
+constexpr int kSampleThreads = 1024;  // threads of a sample CTA (4 samples each)
 constexpr int kSampleRun = 8;  // adjacent positions per sampled run (one 256-byte read at r = 32 FP8)
 
 // Position of sample j of S (S = min(n, kSampleMax)): every position when n <= kSampleMax, else runs
@@ -397,8 +397,7 @@ __device__ __forceinline__ int sample_pos(int j, int n) {
   return (int)(((uint32_t)(j / kSampleRun) * (uint32_t)n) >> 9) + (j % kSampleRun);
 }
 
-// MINB: CTAs per SM the launch is built for (2 for the B*T index rows of the multi-query top-M,
-// which then loads its sampled rows in two batches).
+// MINB: CTAs per SM the launch is built for (with MINB > 1 the sampled rows load in batches of 4).
 template <int R, bool FP8, int MINB = 1>
 __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel(IndexParams p) {
   __shared__ float qbar[128];
@@ -1138,7 +1137,7 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
 // of the projected keys for all T tokens of each sequence.
 template <int R>
 static cudaError_t launch_topm_multi_t(const IndexParams& p, const MultiParams& m, cudaStream_t stream) {
-  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true, 2>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
+  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
   e = launch_index_topm_multi_stream(m, stream);
   if (e != cudaSuccess) return e;
