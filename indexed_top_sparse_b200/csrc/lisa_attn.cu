@@ -8,10 +8,11 @@
 // voor efficiëntie") are applied where the partitions of a (sequence, KV head) are merged.
 //
 // Design on B200:
-//  * Stream-K over the flattened (sequence x KV head, 64-position tile) space: a fixed grid of
-//    CTAs, each taking an equal contiguous run of tiles, so every SM streams for the whole kernel
-//    with one pipeline fill, whatever the batch.  A CTA whose run crosses into the next
-//    (sequence, KV head) writes a partial (max, sum, unnormalised output) for the part it covered.
+//  * Stream-K over the flattened (sequence x KV head, 64-position tile) space: a grid of CTAs (at
+//    most two per SM, chosen on the host so that runs end on (sequence, KV head) boundaries where
+//    the tile counts allow), each taking an equal contiguous run of tiles, so every SM streams for
+//    the whole kernel with one pipeline fill, whatever the batch.  A CTA writes a partial (max,
+//    sum, unnormalised output) for each (sequence, KV head) part it covered.
 //  * The CTA first resolves the pool rows of all its positions (at most kAttnMaxTiles tiles) through
 //    the page table, all index loads then all page loads in flight together; then 64 K rows and 64 V
 //    rows per tile (256 B each at d = 128) are copied with 16-byte cp.async into a 3-stage ring
