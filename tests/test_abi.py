@@ -53,6 +53,22 @@ def test_workspace_size_and_splits():
     assert L.lisa_num_splits(big) >= 16
 
 
+def test_attention_grid_follows_pair_boundaries():
+    # partial slots per pair = parts per pair + 1; the parts divide the 64-position tiles of a pair
+    # when the grid has room (at most 296 CTAs), and no part exceeds 16 tiles
+    big = dict(max_seq_len=131072, max_pages_per_seq=2048, num_pages=32768)
+    cases = [
+        (dict(batch=16, num_q_heads=64, num_kv_heads=8, budget_m=2048), 2),   # 128 pairs x 32 tiles
+        (dict(batch=4, num_q_heads=64, num_kv_heads=8, budget_m=2048), 8),    # 32 pairs: 296 // 32 = 9 -> 8
+        (dict(batch=1, num_q_heads=64, num_kv_heads=8, budget_m=2048), 32),   # 8 pairs: one tile each
+        (dict(batch=32, num_q_heads=64, num_kv_heads=8, budget_m=2048), 2),   # 256 pairs: 16 tiles per part
+        (dict(batch=64, num_q_heads=32, num_kv_heads=8, budget_m=4096), 4),   # 512 pairs x 64 tiles
+    ]
+    for kw, parts in cases:
+        d = _desc(**big, **kw)
+        assert L.lisa_num_splits(d) == parts + 1, (kw, L.lisa_num_splits(d))
+
+
 @pytest.mark.parametrize(
     "kw,status",
     [
