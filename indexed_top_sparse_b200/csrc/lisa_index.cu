@@ -397,9 +397,12 @@ __device__ __forceinline__ int sample_pos(int j, int n) {
   return (int)(((uint32_t)(j / kSampleRun) * (uint32_t)n) >> 9) + (j % kSampleRun);
 }
 
-// MINB: CTAs per SM the launch is built for (with MINB > 1 the sampled rows load in batches of 4).
-template <int R, bool FP8, int MINB = 1>
-__global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel(IndexParams p) {
+// THREADS: threads per CTA (kSampleMax / THREADS samples each); MINB: CTAs per SM the launch is
+// built for (with MINB > 1 the sampled rows load in batches of 4).  The decode step runs one
+// 1024-thread CTA per (b, KV head); the multi-query top-M, with T times the index rows, two
+// 512-thread CTAs per SM.
+template <int R, bool FP8, int THREADS = kSampleThreads, int MINB = 1>
+__global__ void __launch_bounds__(THREADS, MINB) lisa_index_sample_kernel(IndexParams p) {
   __shared__ float qbar[128];
   __shared__ float u[32];
   __shared__ uint32_t hist[kBins];
@@ -407,8 +410,8 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   __shared__ uint32_t scan[32];
   __shared__ uint32_t digit[2];
   using Geo = RowGeom<R, FP8>;
-  constexpr int SPT = kSampleMax / kSampleThreads;  // samples per thread
-  constexpr int kPW = 32 / (kSampleThreads / 32);   // rows of P per warp (r <= 32)
+  constexpr int SPT = kSampleMax / THREADS;  // samples per thread
+  constexpr int kPW = 32 / (THREADS / 32);   // rows of P per warp (r <= 32)
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t bh = (size_t)b * p.Hkv + h;
   pdl_wait();  // first kernel of the step: everything it reads may come from earlier stream work
@@ -431,7 +434,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   float prow[kPW][4];  // P[h][warp + 16 w][lane + 32 i]
 #pragma unroll
   for (int w = 0; w < kPW; ++w) {
-    const int j = warp + (kSampleThreads / 32) * w;
+    const int j = warp + (THREADS / 32) * w;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int c = lane + 32 * i;
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   int pg[SPT], tpos[SPT];
 #pragma unroll
   for (int k = 0; k < SPT; ++k) {
-    const int j = tid + k * kSampleThreads;
+    const int j = tid + k * THREADS;
     pg[k] = 0;
     tpos[k] = sample_pos(j, n);
     if (sampling && j < S) pg[k] = p.page_table[(size_t)bs * p.max_pages + (tpos[k] >> p.log2ps)];
@@ -457,7 +460,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   auto load_batch = [&](int k0) {
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
-      const int j = tid + (k0 + k) * kSampleThreads;
+      const int j = tid + (k0 + k) * THREADS;
       if (sampling && j < S) {
         const int t = tpos[k0 + k];
         int pgk = pg[k0 + k];
@@ -476,7 +479,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   __syncthreads();
 #pragma unroll
   for (int wr = 0; wr < kPW; ++wr) {
-    const int j = warp + (kSampleThreads / 32) * wr;
+    const int j = warp + (THREADS / 32) * wr;
     float acc = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -509,7 +512,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
     if (k0 > 0) load_batch(k0);
 #pragma unroll
     for (int k = 0; k < KB; ++k) {
-      const int j = tid + (k0 + k) * kSampleThreads;
+      const int j = tid + (k0 + k) * THREADS;
       if (j < S) {
         const uint32_t key = score_key(scale * row_dot<R, FP8>(w[k], u2));
         skey[j] = key;
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(kSampleThreads, MINB) lisa_index_sample_kernel
   }
   if (bad) flag_error(p.err, bad);
   __syncthreads();
-  const uint32_t tau = sample_threshold<kSampleThreads>(hist, skey, S, n, p.M, scan, digit);
+  const uint32_t tau = sample_threshold<THREADS>(hist, skey, S, n, p.M, scan, digit);
   if (tid == 0) p.tau[bh] = tau;
 }
 
@@ -1137,7 +1140,7 @@ static cudaError_t launch_topm_t(const IndexParams& p, cudaStream_t stream, cuda
 // of the projected keys for all T tokens of each sequence.
 template <int R>
 static cudaError_t launch_topm_multi_t(const IndexParams& p, const MultiParams& m, cudaStream_t stream) {
-  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true>, dim3(p.Hkv, p.B), dim3(kSampleThreads), 0, stream, p);
+  cudaError_t e = launch_pdl(lisa_index_sample_kernel<R, true, 512, 2>, dim3(p.Hkv, p.B), dim3(512), 0, stream, p);
   if (e != cudaSuccess) return e;
   e = launch_index_topm_multi_stream(m, stream);
   if (e != cudaSuccess) return e;
