@@ -1,0 +1,36 @@
+"""CPU checks of bench.py's host-side bookkeeping (no GPU): the recorded DRAM traffic of the score
+stream kernel is reported only while the kernel sources are the ones it was captured from."""
+
+import importlib.util
+import json
+import os
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_committed_traffic_record_matches_the_sources():
+    b = _bench()
+    rec = json.load(open(b.TRAFFIC_FILE))
+    assert rec["source_hash"] == b.source_hash(b.INDEX_SOURCES)
+    t = b.recorded_traffic()
+    assert t == rec["dram_bytes_per_launch_full_workload"]
+    # scaled from the captured launches, and close to (not below) the algorithmic bytes
+    mean = sum(l["dram_bytes_read"] + l["dram_bytes_write"] for l in rec["captured_launches"]) / len(
+        rec["captured_launches"])
+    assert abs(t - mean * rec["scale_to_full_workload"]) < 1.0
+    assert 1.0 <= t / rec["algorithmic_bytes_per_launch_full_workload"] < 1.05
+
+
+def test_traffic_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch):
+    b = _bench()
+    changed = tmp_path / "lisa_index.cu"
+    changed.write_bytes(open(os.path.join(ROOT, b.INDEX_SOURCES[0]), "rb").read() + b"\n// edited\n")
+    monkeypatch.setattr(b, "INDEX_SOURCES", [str(changed)] + list(b.INDEX_SOURCES[1:]))
+    assert b.recorded_traffic() is None
