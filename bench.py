@@ -358,6 +358,13 @@ def run_ours(args, world, rank, local):
     inplace_ms = dev_time(lambda: L.lisa_sparse_decode_attn(desc, prob.q, k_arg, v_arg, idx_c, cnt_c, out, lse, ws,
                                                             stream=stream), max(3, min(K, 50)))
     del gta, dense_ws
+    # Scores only (lisa_index_score): the fp32 score of every position, for callers that select
+    # themselves; the fused path never writes them.
+    sc_all = torch.empty(B, prob.Hkv, prob.max_seq_len, dtype=torch.float32, device=dev)
+    score_ms = dev_time(lambda: L.lisa_index_score(desc, prob.q, prob.P, prob.kproj, L.KPROJ_FP8_E4M3, scale, sc_all, ws,
+                                                   stream=stream), max(3, min(K, 20)))
+    score_bytes = float(sum(int(n) * prob.r * prob.Hkv for n in prob.seq_lens.tolist()) + sc_all.numel() * 4)
+    del sc_all
     # Multi-query indexer (speculative decoding with 4 draft tokens per sequence): the scores of all
     # positions for every token, the 4 projected queries forming one tensor-core contraction.
     Tq = 4
@@ -462,6 +469,12 @@ def run_ours(args, world, rank, local):
             "gather_share_of_gather_then_attend": gather_ms / (gather_ms + attend_ms),
             "in_place_attention_ms": inplace_ms,
             "gather_then_attend_over_in_place": (gather_ms + attend_ms) / inplace_ms,
+        },
+        "index_scores_only": {
+            "entry": "lisa_index_score (fp32 score of every position written)",
+            "ms_per_call": score_ms,
+            "bytes_per_call": score_bytes,
+            "achieved_gbs": score_bytes / (score_ms * 1e-3) / 1e9,
         },
         "multi_query_index_scores": {
             "entry": "lisa_index_score_multi",

@@ -194,6 +194,34 @@ IndexParams index_params(const lisa_decode_desc& d, const Layout& L, void* ws) {
   return p;
 }
 
+// Launch parameters of the multi-query score stream for T tokens per sequence (scores mode).
+MultiParams multi_params(const lisa_decode_desc& d, const Layout& L, int T, const void* q, const float* P,
+                         const void* kproj_pool, const float* kproj_scale, float* scores, void* ws) {
+  MultiParams p{};
+  p.B = d.batch;
+  p.T = T;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.d = d.head_dim;
+  p.r = d.idx_dim;
+  p.ps = d.page_size;
+  p.log2ps = ilog2(d.page_size);
+  p.max_pages = d.max_pages_per_seq;
+  p.max_seq_len = d.max_seq_len;
+  p.num_pages = d.num_pages;
+  p.seq_lens = d.seq_lens;
+  p.page_table = d.page_table;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.P = P;
+  p.kproj = kproj_pool;
+  p.kproj_scale = kproj_scale;
+  p.scores = scores;
+  // the projected queries go where the fused top-M keeps its candidates (room for kMultiMaxT tokens)
+  p.uq = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.off_cand);
+  p.err = static_cast<uint32_t*>(ws);
+  return p;
+}
+
 AttnParams attn_params(const lisa_decode_desc& d, const Layout& L, void* ws, const void* q, const void* k_pool,
                        const void* v_pool, const int32_t* idx, const int32_t* count, void* out, float* lse,
                        const lisa_linear_branch* lin) {
@@ -349,11 +377,17 @@ lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const 
   const Layout L = layout_of(*desc);
   LISA_TRY(check_ws(ws, ws_bytes, L));
   LISA_TRY(bind_device(ws));
+  if (kproj_dtype == LISA_KPROJ_FP8_E4M3) {
+    // FP8 keys: the tensor-core score stream of the multi-query indexer with one token, which sees
+    // every position t < n_b and writes scores[b][0][h][t] = scores[b][h][t].
+    const MultiParams m = multi_params(*desc, L, 1, q, P, kproj_pool, kproj_scale, scores, ws);
+    return cuda_status(launch_index_score_multi(m, reinterpret_cast<cudaStream_t>(stream)));
+  }
   IndexParams p = index_params(*desc, L, ws);
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.P = P;
   p.kproj = kproj_pool;
-  p.kproj_fp8 = kproj_dtype == LISA_KPROJ_FP8_E4M3;
+  p.kproj_fp8 = false;
   p.kproj_scale = kproj_scale;
   p.scores = scores;
   return cuda_status(launch_index_score(p, reinterpret_cast<cudaStream_t>(stream)));
@@ -373,27 +407,7 @@ lisa_status lisa_index_score_multi(const lisa_decode_desc* desc, int num_tokens,
   const Layout L = layout_of(*desc);
   LISA_TRY(check_ws(ws, ws_bytes, L));
   LISA_TRY(bind_device(ws));
-  MultiParams p{};
-  p.B = desc->batch;
-  p.T = num_tokens;
-  p.Hq = desc->num_q_heads;
-  p.Hkv = desc->num_kv_heads;
-  p.d = desc->head_dim;
-  p.r = desc->idx_dim;
-  p.ps = desc->page_size;
-  p.log2ps = ilog2(desc->page_size);
-  p.max_pages = desc->max_pages_per_seq;
-  p.max_seq_len = desc->max_seq_len;
-  p.num_pages = desc->num_pages;
-  p.seq_lens = desc->seq_lens;
-  p.page_table = desc->page_table;
-  p.q = static_cast<const __nv_bfloat16*>(q);
-  p.P = P;
-  p.kproj = kproj_pool;
-  p.kproj_scale = kproj_scale;
-  p.scores = scores;
-  p.uq = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.off_cand);
-  p.err = static_cast<uint32_t*>(ws);
+  const MultiParams p = multi_params(*desc, L, num_tokens, q, P, kproj_pool, kproj_scale, scores, ws);
   return cuda_status(launch_index_score_multi(p, reinterpret_cast<cudaStream_t>(stream)));
 }
 
