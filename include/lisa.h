@@ -147,7 +147,9 @@ int32_t lisa_num_splits(const lisa_decode_desc* desc);
 /* Zero the workspace error word (enqueued on stream). Call once after allocating ws. */
 lisa_status lisa_workspace_init(void* ws, size_t ws_bytes, lisa_stream_t stream);
 
-/* Steps 1-3: write s_t to scores[b][h][t] for t < n_b (entries t >= n_b are not written). */
+/* Steps 1-3: write s_t to scores[b][h][t] for t < n_b (entries t >= n_b are not written).  With
+ * FP8 projected keys this is lisa_index_score_multi with one token per sequence (same kernels, same
+ * use of ws); with fp32 keys one CUDA-core kernel. */
 lisa_status lisa_index_score(const lisa_decode_desc* desc, const void* q, const float* P,
                              const void* kproj_pool, lisa_kproj_dtype kproj_dtype,
                              const float* kproj_scale, float* scores, void* ws, size_t ws_bytes,
