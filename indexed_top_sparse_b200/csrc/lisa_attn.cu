@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   // tiles of the pipeline prologue all sit in slot 0.
   static_assert((kAttnStages - 1) * kAttnTile <= kAttnThreads, "prologue tiles must fit in slot 0");
 
-  // Round 1: the count and sequence length of each touched pair, and the index of every slot (address
+  // Load round 1: the count and sequence length of each touched pair, and the index of every slot (address
   // clamped into the pair's M entries, validity applied later), all in flight together.
   if (tid == 0) s_last = 0u;
   uint32_t bad = 0u;  // LISA_DEVERR_* bits seen by this thread, flagged once at the end of the prologue
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) lisa_sparse_attn_kernel(AttnP
   }
   __syncthreads();
 
-  // Round 2: page-table loads of slots [k0, k1), then their pool rows (row = (page * ps + slot) *
+  // Load round 2: page-table loads of slots [k0, k1), then their pool rows (row = (page * ps + slot) *
   // Hkv + h, or kNoRow past the pair's count) into rows_sm.
   auto resolve = [&](auto k0c, auto k1c) {
     constexpr int k0 = decltype(k0c)::value, k1 = decltype(k1c)::value;
